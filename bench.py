@@ -1,0 +1,401 @@
+#!/usr/bin/env python3
+"""Benchmark of the CSA decode step (the hot path of the compressed sparse attention).
+
+Workload (one attention layer, one decode step = one new token for each of B
+requests): CSA decode, bf16 -- 32 requests with a 128K-token context each:
+32768 compressed entries (m = 4) of dim 576 (512 content + 64 RoPE), 64 query
+heads sharing the KV, lightning indexer with 64 heads x 128 dims over bf16 keys,
+top-512 selection, a 128-row raw window; values N(0,1), query scale 1/sqrt(576).
+A step runs the whole path (index scoring -> top-k -> sparse MQA) through
+decode_fused.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 is launched with torchrun: every rank runs its own batch of 32 requests on
+its own GPU (requests are independent: no collective on the data path); the
+step time is the max over ranks.  One JSON line is printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA decode tok/s and achieved HBM GB/s vs roofline at 128K-1M ctx"
+UNIT = "tok/s"
+WORKLOAD = dict(workload="csa_decode_bf16_128k", requests=32, context_tokens=131072, compressed_entries=32768,
+                m=4, kv_dim=576, d_v=512, heads=64, index_heads=64, index_dim=128, topk=512, window=128)
+B, NC, D, DV, H, HI, DI, K, TW = 32, 32768, 576, 512, 64, 64, 128, 512, 128
+SCALE = 1.0 / math.sqrt(576.0)
+
+
+def algorithmic_bytes_per_request():
+    keys = NC * DI * 2
+    sel = K * D * 2
+    win = TW * D * 2
+    qin = H * D * 2 + HI * DI * 2 + HI * 4
+    out = H * DV * 2
+    return keys + sel + win + qin + out
+
+
+def index_bytes_per_request():
+    return NC * DI * 2 + HI * DI * 2 + HI * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+INDEX_KERNEL_FILES = ["long_context_sparse_06_b200/csrc/indexer.cu", "long_context_sparse_06_b200/csrc/lcs_common.cuh"]
+
+
+def recorded_traffic(kernel):
+    """dram bytes per launch from a committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_hash") != kernel_source_hash(INDEX_KERNEL_FILES):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+               0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(device_index)
+            pci = getattr(bus, "pci_bus_id", None)
+            if pci is not None:
+                dom = getattr(bus, "pci_domain_id", 0)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{pci:02x}:{getattr(bus, 'pci_device_id', 0):02x}.0")
+            else:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                idx = int(vis.split(",")[device_index]) if vis else device_index
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+        except Exception:
+            self._h = None
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        for bit, name in self.REASONS.items():
+            if r & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            self._stop.wait(0.01)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ inputs
+def make_inputs(device, rank):
+    import torch
+    from long_context_sparse_06_b200 import synth
+    tag = f"bench.r{rank}."
+    bf = torch.bfloat16
+    x = dict(
+        q=synth.normal_t(tag + "q", (B, H, D), dtype=bf, device=device),
+        comp=synth.normal_t(tag + "comp", (B, NC, D), dtype=bf, device=device),
+        win=synth.normal_t(tag + "win", (B, TW, D), dtype=bf, device=device),
+        qI=synth.normal_t(tag + "qI", (B, HI, DI), dtype=bf, device=device),
+        w=synth.normal_t(tag + "w", (B, HI), std=1.0 / 8, dtype=torch.float32, device=device),
+        kI=synth.normal_t(tag + "kI", (B, NC, DI), dtype=bf, device=device),
+    )
+    return x
+
+
+# ------------------------------------------------------------------- arms
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import long_context_sparse_06_b200 as lcs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lcs.lib()
+
+    x = make_inputs(dev, rank)
+    out = torch.empty((B, H, DV), dtype=torch.bfloat16, device=dev)
+    ws = lcs.workspace(lcs.lcs_workspace_size(lcs.OP_DECODE, B, 1, NC, TW, K, H, DV, lcs.F32), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lcs.decode_fused(lcs.MODE_CSA, x["q"], x["comp"], x["win"], DV, SCALE, qI=x["qI"], w=x["w"], kI=x["kI"],
+                         k=K, out=out, ws=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = lcs.lcs_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {st}")
+
+    # ---- timed region: K steps of the whole path, inputs (297 MB/step) larger than L2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms_total / args.steps
+    value = world * B / (ms_step / 1e3)
+
+    # ---- per-stage device time of the same steps (events on the launching stream)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    handles = (lcs.C.c_void_p * 4)(*[e.cuda_event for e in evs])
+    stage_ms = [0.0, 0.0, 0.0]
+    lcs.lib().lcs_set_stage_events(handles, 4)
+    try:
+        for _ in range(args.steps):
+            step()
+            torch.cuda.synchronize()
+            for i in range(3):
+                stage_ms[i] += evs[i].elapsed_time(evs[i + 1])
+    finally:
+        lcs.lib().lcs_set_stage_events(None, 0)
+    stage_ms = [s / args.steps for s in stage_ms]
+    stage_ms = [max_over_ranks(s) for s in stage_ms]
+
+    # ---- end to end through the public API: per-step inputs H2D from pinned host, result D2H
+    hq = x["q"].cpu().pin_memory()
+    hqI = x["qI"].cpu().pin_memory()
+    hw = x["w"].cpu().pin_memory()
+    hwin_row = x["win"][:, -1].contiguous().cpu().pin_memory()
+    hout = torch.empty((B, H, DV), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hqI, hw, hwin_row))
+    d2h = hout.numel() * hout.element_size()
+    win_last = x["win"][:, -1]
+
+    def e2e_step():
+        x["q"].copy_(hq, non_blocking=True)
+        x["qI"].copy_(hqI, non_blocking=True)
+        x["w"].copy_(hw, non_blocking=True)
+        win_last.copy_(hwin_row, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    st = lcs.lcs_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {st}")
+
+    peak, peak_kind = load_peaks()
+    idx_bytes = B * index_bytes_per_request()
+    achieved = idx_bytes / (stage_ms[0] / 1e3) / 1e9
+    step_bytes = B * algorithmic_bytes_per_request()
+    res = None
+    if rank == 0:
+        cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline(x)
+        res = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))",
+            "config": dict(WORKLOAD, l2="inputs larger than L2 (297 MB/step vs 126 MB)",
+                           parallelism=f"replicas x{world} (requests independent)"),
+            "roofline": {"bound": "hbm", "kernel": "index_bf16_tc_kernel", "achieved": round(achieved, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": idx_bytes,
+                         "traffic": recorded_traffic("index_bf16_tc_kernel")},
+            "step_roofline": {"algorithmic_bytes_per_step": step_bytes,
+                              "achieved_gbs": round(step_bytes / (ms_step / 1e3) / 1e9, 1),
+                              "frac": round(step_bytes / (ms_step / 1e3) / 1e9 / peak, 4)},
+            "stage_ms": {"index": round(stage_ms[0], 5), "topk": round(stage_ms[1], 5),
+                         "attend": round(stage_ms[2], 5)},
+            "e2e": {"value": round(world * B / (e2e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
+                    "inputs": "per-step q, qI, w and the new window row from pinned host; caches resident"},
+            "gpu_launches": args.steps * 4,
+            "clocks": sampler.summary(),
+            "cpu_baseline": cpu,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return res
+
+
+def cpu_baseline(x, budget_s=20.0):
+    """The oracle, as it stands, on a bounded sample of the same workload: whole
+    requests, in order, until about budget_s seconds of oracle compute."""
+    from oracle import oracle as orc
+    el, n = 0.0, 0
+    while n < B and el < budget_s:
+        qI = x["qI"][n].double().cpu().numpy()
+        kI = x["kI"][n].double().cpu().numpy()
+        w = x["w"][n].cpu().numpy()
+        q = x["q"][n].double().cpu().numpy()
+        win = x["win"][n].double().cpu().numpy()
+        comp = x["comp"][n].double().cpu().numpy()
+        ts = time.perf_counter()
+        s = orc.index_scores_bf16(qI, w, kI)
+        idx = orc.topk(s, K)
+        orc.csa_attend(q, comp, idx, win, 0, -1, TW, DV, SCALE)
+        el += time.perf_counter() - ts
+        n += 1
+    return {"value": round(n / el, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {B} requests of the same workload, full path per request (index over all "
+                      f"{NC} entries, top-{K}, attention over {K}+{TW} rows); single thread"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import numpy as np
+    import torch
+    from long_context_sparse_06_b200 import synth
+    from oracle import oracle as orc
+    # per-step sample: one request; the indexer over a contiguous slice of the entries,
+    # extrapolated to all NC entries; top-k and attention in full
+    total_budget = 150.0
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    probe = 2048
+    bf = torch.bfloat16
+    qI = synth.normal_t("ref.qI", (HI, DI), dtype=bf).double().numpy()
+    w = synth.normal_t("ref.w", (HI,), std=1.0 / 8).numpy()
+    kI = synth.normal_t("ref.kI", (NC, DI), dtype=bf).double().numpy()
+    q = synth.normal_t("ref.q", (H, D), dtype=bf).double().numpy()
+    comp = synth.normal_t("ref.comp", (NC, D), dtype=bf).double().numpy()
+    win = synth.normal_t("ref.win", (TW, D), dtype=bf).double().numpy()
+    t = time.perf_counter()
+    orc.index_scores_bf16(qI, w, kI[:probe])
+    per_key = (time.perf_counter() - t) / probe
+    n_slice = int(min(NC, max(probe, (per_step * 0.8) / per_key)))
+
+    def one_step():
+        t0 = time.perf_counter()
+        s = orc.index_scores_bf16(qI, w, kI[:n_slice])
+        t_index = (time.perf_counter() - t0) * (NC / n_slice)
+        full = np.full(NC, -np.inf, np.float32)
+        full[:n_slice] = s
+        t1 = time.perf_counter()
+        idx = orc.topk(full, K)
+        orc.csa_attend(q, comp, idx, win, 0, -1, TW, DV, SCALE)
+        return t_index + (time.perf_counter() - t1)
+
+    for _ in range(args.warmup):
+        one_step()
+    total = sum(one_step() for _ in range(args.steps))
+    ms = total / args.steps * 1e3
+    value = 1.0 / (ms / 1e3)
+    sample = (f"1 request per step; indexer over {n_slice} of {NC} entries, time scaled to all entries; "
+              f"top-{K} and attention over {K}+{TW} rows in full; single thread")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 where the oracle fixes it)",
+            "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))", "config": dict(WORKLOAD),
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(value, 4), "unit": UNIT},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="lcs", choices=["lcs", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

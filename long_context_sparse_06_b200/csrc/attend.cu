@@ -1,0 +1,574 @@
+// attend.cu -- shared-KV MQA over a gathered row set (CSA sparse; HCA dense).
+//
+// "DeepSeek V4 深度解析" §2, CSA step 3: the selected compressed entries and the
+// most recent 128 raw tokens are attended together; HCA paragraph: dense
+// attention over every compressed entry plus the window; both use shared-KV
+// multi-query attention.  For query (b,q) and head h:
+//   o_h = sum_r softmax_r(scale * q_h . K_r) V_r,  V_r = first d_v dims of K_r,
+// one softmax over the union of the selected (or all available) compressed
+// rows and the window rows.
+//
+// Tensor-core path (H = 64, D = 576, d_v = 512; bf16 rows or FP8 rows):
+//  * one CTA per (query, split of its row list), rows processed in chunks of 64;
+//  * warp 8 loads the 64 query heads once (TMA, 128-byte swizzle) and issues
+//    tcgen05.mma with the query heads as M = 64:
+//      S [64 heads x 64 rows] = Q [64 x 576] . K_chunk^T        (K-major x K-major)
+//      O [64 heads x 512]    += P [64 x 64 rows] . V_chunk       (K-major x MN-major)
+//    O lives in TMEM as two interleaved M=64 accumulators (dims 0-255 in lanes
+//    0-15 of each 32-lane quarter, dims 256-511 in lanes 16-31), S beside it;
+//  * warps 4-7 gather the chunk's rows into a 2-stage ring with 16-byte
+//    cp.async (bf16) or load-convert-store (FP8 rows: E4M3 x block scale ->
+//    bf16), writing the SW128 layout that both MMAs read (the same bytes are
+//    the K-major B of Q.K^T and the MN-major B of P.V);
+//  * warps 0-3 run the online softmax on S (fp32, exp2), write P as bf16 into
+//    the chunk's RoPE column block (dead once Q.K^T has read it), rescale O in
+//    TMEM only when a head's running max grows by more than 2^8 in weight, and
+//    finally normalise O and write it out (or a split partial for the combine).
+// F32 path (C1-sized problems): CUDA cores, fp32 online softmax.
+#include <utility>
+
+#include "lcs_common.cuh"
+#include "lcs_internal.h"
+
+namespace lcs {
+
+namespace {
+
+constexpr int kH = 64, kD = 576, kDv = 512, kChunk = 64;
+constexpr int kBlk = kChunk * 128;            // one SW128 column block of a chunk: 64 rows x 128 B
+constexpr int kStageBytes = 9 * kBlk;         // 72 KB
+constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
+constexpr int kMaxK = 2048;
+constexpr int kAtThreads = 288;
+constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kMaxK * 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
+
+struct AtBars {
+    uint64_t qfull;
+    uint64_t kfull[2], kempty[2];
+    uint64_t sfull, sempty;
+    uint64_t pfull[2];
+    uint64_t ofull;
+    uint32_t tmem_base;
+    int nsel;
+};
+
+struct RowPlan {
+    int64_t nsel;        // selected / available compressed rows
+    int64_t win_lo;      // first window row index in win[b]
+    int64_t nwin;
+};
+
+__device__ __forceinline__ RowPlan plan_rows(const AttendArgs& a, int64_t g, int nsel) {
+    RowPlan p;
+    const int64_t b = g / a.Q;
+    p.nsel = nsel;
+    if (a.q_pos == nullptr) {
+        p.win_lo = 0;
+        p.nwin = a.Tw;
+    } else {
+        const int64_t t = a.q_pos[g];
+        const int64_t wp0 = a.win_pos0[b];
+        int64_t lo = t - a.W + 1 - wp0, hi = t - wp0;
+        if (lo < 0) lo = 0;
+        if (hi > a.Tw - 1) hi = a.Tw - 1;
+        p.win_lo = lo;
+        p.nwin = hi >= lo ? hi - lo + 1 : 0;
+    }
+    return p;
+}
+
+// Row pointer of row position r of query g (bf16 rows: D elements; FP8: 656 B).
+__device__ __forceinline__ const uint8_t* row_ptr(const AttendArgs& a, int64_t b, const RowPlan& p,
+                                                  const int* sel, int64_t r, int row_bytes) {
+    if (r < p.nsel) {
+        const int64_t e = sel ? sel[r] : r;
+        return static_cast<const uint8_t*>(a.comp) + (b * a.N_c + e) * row_bytes;
+    }
+    return static_cast<const uint8_t*>(a.win) + (b * a.Tw + p.win_lo + (r - p.nsel)) * row_bytes;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kAtThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const AttendArgs a, int splits,
+                     float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ AtBars bars;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* q_s = smem;
+    uint8_t* stage_s = smem + kQBytes;
+    int* sel_s = reinterpret_cast<int*>(smem + kQBytes + 2 * kStageBytes);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t g = blockIdx.x / splits;
+    const int sp = blockIdx.x - (int)(g * splits);
+    const int64_t b = g / a.Q;
+    constexpr int row_bytes = FP8 ? 656 : kD * 2;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars.qfull, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars.kfull[i], 128);
+            mbar_init(&bars.kempty[i], 1);
+            mbar_init(&bars.pfull[i], 128);
+        }
+        mbar_init(&bars.sfull, 1);
+        mbar_init(&bars.sempty, 128);
+        mbar_init(&bars.ofull, 1);
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(&bars.tmem_base, 512);
+        tmem_relinquish();
+    }
+#if defined(__CUDA_ARCH__)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+    // ---- selection list (CSA: valid entries of idx in order; HCA: implicit)
+    if (a.idx != nullptr) {
+        if (warp == 0) {
+            const int32_t* ir = a.idx + g * a.k;
+            int cnt = 0;
+            for (int base = 0; base < a.k; base += 32) {
+                const int i = base + lane;
+                int32_t v = (i < a.k) ? ir[i] : -1;
+                if (v >= a.N_c) { set_status(status, LCS_ERR_DEVICE, 201); v = -1; }
+                const bool ok = v >= 0;
+                const uint32_t bal = __ballot_sync(0xffffffffu, ok);
+                if (ok) sel_s[cnt + __popc(bal & ((1u << lane) - 1u))] = v;
+                cnt += __popc(bal);
+            }
+            if (lane == 0) bars.nsel = cnt;
+        }
+    } else if (threadIdx.x == 0) {
+        int64_t n = a.N_c;
+        if (a.q_pos != nullptr) {
+            const int64_t av = (a.q_pos[g] + 1) / a.m;
+            n = av < 0 ? 0 : (av < a.N_c ? av : a.N_c);
+        }
+        bars.nsel = (int)n;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+    const int* sel = (a.idx != nullptr) ? sel_s : nullptr;
+    const RowPlan plan = plan_rows(a, g, bars.nsel);
+    const int64_t R = plan.nsel + plan.nwin;
+    const int64_t nch_all = (R + kChunk - 1) / kChunk;
+    const int64_t cps = (nch_all + splits - 1) / splits;
+    const int64_t c_begin = sp * cps;
+    const int64_t c_end = (c_begin + cps < nch_all) ? c_begin + cps : nch_all;
+    const int nch = (int)(c_end > c_begin ? c_end - c_begin : 0);
+
+    constexpr uint32_t idesc_qk = idesc_bf16(64, kChunk, false, false);
+    constexpr uint32_t idesc_pv = idesc_bf16(64, 256, false, true);
+    const uint32_t t_s = tmem + 256;   // S: columns 256..319, lanes of the M=64 layout
+
+    if (warp == 8) {
+        if (lane == 0 && nch > 0) {
+            // ---------------- Q load + MMA issue
+            mbar_arrive_expect_tx(&bars.qfull, kQBytes);
+            for (int blk = 0; blk < 9; ++blk)
+                tma_load_2d(q_s + blk * (kH * 128), &map_q, &bars.qfull, blk * 64, (int)(g * kH));
+            bool ok = mbar_wait(&bars.qfull, 0, status, 300);
+            const uint32_t q_base = smem_u32(q_s);
+            auto issue_qk = [&](int c) -> bool {
+                const int st = c & 1;
+                if (!mbar_wait(&bars.kfull[st], (uint32_t)((c >> 1) & 1), status, 301)) return false;
+                if (c > 0 && !mbar_wait(&bars.sempty, (uint32_t)((c - 1) & 1), status, 302)) return false;
+                tc_fence_after();
+                const uint32_t k_base = smem_u32(stage_s + st * kStageBytes);
+                for (int blk = 0; blk < 9; ++blk)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = sw128_desc(q_base + blk * (kH * 128) + kk * 32, 16, 1024);
+                        const uint64_t bd = sw128_desc(k_base + blk * kBlk + kk * 32, 16, 1024);
+                        mma_bf16_ss(t_s, ad, bd, idesc_qk, (blk | kk) ? 1u : 0u);
+                    }
+                mma_commit(&bars.sfull);
+                return true;
+            };
+            if (ok) ok = issue_qk(0);
+            for (int c = 0; c < nch && ok; ++c) {
+                if (c + 1 < nch) ok = issue_qk(c + 1);
+                if (!ok) break;
+                const int st = c & 1;
+                if (!mbar_wait(&bars.pfull[st], (uint32_t)((c >> 1) & 1), status, 303)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t p_base = smem_u32(stage_s + st * kStageBytes + 8 * kBlk);
+                const uint32_t v_base = smem_u32(stage_s + st * kStageBytes);
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = sw128_desc(p_base + kk * 32, 16, 1024);
+                        const uint64_t bd = sw128_desc(v_base + half * 4 * kBlk + kk * 2048, kBlk, 1024);
+                        mma_bf16_ss(tmem + (half ? (16u << 16) : 0u), ad, bd, idesc_pv, (c | kk) ? 1u : 0u);
+                    }
+                mma_commit(&bars.kempty[st]);
+                mma_commit(&bars.ofull);
+            }
+        }
+    } else if (warp >= 4) {
+        // ---------------- gather producer: warps 4..7 (128 threads)
+        const int pt = threadIdx.x - 128;
+        for (int c = 0; c < nch; ++c) {
+            const int st = c & 1;
+            if (c >= 2 && !mbar_wait(&bars.kempty[st], (uint32_t)(((c - 2) >> 1) & 1), status, 310)) break;
+            uint8_t* dst = stage_s + st * kStageBytes;
+            const int64_t r0 = (c_begin + c) * kChunk;
+            if constexpr (!FP8) {
+                // 64 rows x 72 chunks of 16 B; thread pt takes chunks pt, pt+128, ...
+                for (int i = pt; i < kChunk * 72; i += 128) {
+                    const int rr = i / 72, ch = i - rr * 72;
+                    const int64_t r = r0 + rr;
+                    const bool valid = r < R;
+                    const uint8_t* src = valid ? row_ptr(a, b, plan, sel, r, row_bytes) + ch * 16
+                                               : static_cast<const uint8_t*>(a.win);
+                    cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), src, valid);
+                }
+                cp_async_commit();
+                cp_async_wait<0>();
+            } else {
+                // FP8 rows: 32 content segments of 16 codes + 8 RoPE chunks of 8 bf16 per row
+                for (int i = pt; i < kChunk * 40; i += 128) {
+                    const int rr = i / 40, seg = i - rr * 40;
+                    const int64_t r = r0 + rr;
+                    uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+                    if (r < R) {
+                        const uint8_t* src = row_ptr(a, b, plan, sel, r, row_bytes);
+                        if (seg < 32) {
+                            const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + seg * 16));
+                            const float sc = __ldg(reinterpret_cast<const float*>(src + 640) + (seg >> 3));
+                            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                            uint32_t o[8];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                o[2 * q] = pack_bf16x2(e4m3_to_f32(w[q] & 0xFF) * sc, e4m3_to_f32((w[q] >> 8) & 0xFF) * sc);
+                                o[2 * q + 1] =
+                                    pack_bf16x2(e4m3_to_f32((w[q] >> 16) & 0xFF) * sc, e4m3_to_f32(w[q] >> 24) * sc);
+                            }
+                            lo = make_uint4(o[0], o[1], o[2], o[3]);
+                            hi = make_uint4(o[4], o[5], o[6], o[7]);
+                        } else {
+                            lo = __ldg(reinterpret_cast<const uint4*>(src + 512 + (seg - 32) * 16));
+                        }
+                    }
+                    if (seg < 32) {
+                        const int ch = seg * 2;   // two 16-byte bf16 chunks
+                        *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
+                        *reinterpret_cast<uint4*>(dst + ((ch + 1) >> 3) * kBlk + sw128_off(rr, (ch + 1) & 7)) = hi;
+                    } else {
+                        const int ch = 64 + (seg - 32);
+                        *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bars.kfull[st]);
+        }
+    } else {
+        // ---------------- softmax / correction / epilogue: warps 0..3
+        const int quarter = warp;            // TMEM lanes 32*quarter .. +31
+        const int hl = lane & 15;
+        const int head = quarter * 16 + hl;  // head of this thread (both half-rows)
+        const bool lo_half = lane < 16;
+        float m_used = -INFINITY;            // log2-domain running max used for exponentials
+        float l_sum = 0.f;
+        const float sl2 = a.scale * kLog2e;
+        for (int c = 0; c < nch; ++c) {
+            const int st = c & 1;
+            if (!mbar_wait(&bars.sfull, (uint32_t)(c & 1), status, 320)) break;
+            tc_fence_after();
+            uint32_t sv[kChunk];
+#pragma unroll
+            for (int j = 0; j < kChunk / 16; ++j)
+                tmem_ld16(tmem_addr(t_s, quarter * 32, j * 16), *reinterpret_cast<uint32_t(*)[16]>(&sv[j * 16]));
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&bars.sempty);
+            const int64_t rbase = (c_begin + c) * kChunk;
+            const int nvalid = (int)((R - rbase) < kChunk ? (R - rbase) : kChunk);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j)
+                if (j < nvalid) mx = fmaxf(mx, __uint_as_float(sv[j]) * sl2);
+            // lanes 16..31 read the unused upper half-lanes; take the max/decision of lane hl
+            mx = __shfl_sync(0xffffffffu, mx, hl);
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mx > m_used + kRescale || m_used == -INFINITY) {
+                const float m_new = fmaxf(mx, m_used);
+                alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - m_new);
+                rescale = (c > 0);
+                m_used = m_new;
+            }
+            // P (bf16) for this thread's head into the chunk's RoPE block (K-major, 128 B per head row)
+            uint8_t* pblk = stage_s + st * kStageBytes + 8 * kBlk;
+            float psum = 0.f;
+            if (lo_half) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int j0 = ch * 8 + 2 * q;
+                        float p0 = (j0 < nvalid) ? exp2f(__uint_as_float(sv[j0]) * sl2 - m_used) : 0.f;
+                        float p1 = (j0 + 1 < nvalid) ? exp2f(__uint_as_float(sv[j0 + 1]) * sl2 - m_used) : 0.f;
+                        pk[q] = pack_bf16x2(p0, p1);
+                        psum += bf16_bits_to_f32((uint16_t)(pk[q] & 0xFFFF)) + bf16_bits_to_f32((uint16_t)(pk[q] >> 16));
+                    }
+                    *reinterpret_cast<uint4*>(pblk + sw128_off(head, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            l_sum = l_sum * alpha + psum;
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O must be stable: wait for the previous chunk's P.V
+                if (!mbar_wait(&bars.ofull, (uint32_t)((c - 1) & 1), status, 321)) break;
+                tc_fence_after();
+                const float f = rescale ? alpha : 1.f;
+                for (int j = 0; j < 256 / 16; ++j) {
+                    uint32_t ov[16];
+                    const uint32_t ta = tmem_addr(tmem, quarter * 32, j * 16);
+                    tmem_ld16(ta, ov);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * f);
+                    tmem_st16(ta, ov);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bars.pfull[st]);
+        }
+        // ---- epilogue: O / l (or the split partial)
+        const bool have = nch > 0;
+        if (have && !mbar_wait(&bars.ofull, (uint32_t)((nch - 1) & 1), status, 322)) { /* fall through */ }
+        tc_fence_after();
+        const float l_h = __shfl_sync(0xffffffffu, l_sum, hl);
+        const float m_h = __shfl_sync(0xffffffffu, m_used, hl);
+        const int dim0 = lo_half ? 0 : 256;
+        if (splits == 1) {
+            const float inv = (l_h > 0.f) ? 1.f / l_h : 0.f;
+            uint16_t* o = static_cast<uint16_t*>(a.out) + (g * kH + head) * kDv + dim0;
+            for (int j = 0; j < 256 / 16; ++j) {
+                uint32_t ov[16];
+                if (have) {
+                    tmem_ld16(tmem_addr(tmem, quarter * 32, j * 16), ov);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) ov[q] = 0;
+                }
+                uint32_t pk[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    pk[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
+                reinterpret_cast<uint4*>(o + j * 16)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                reinterpret_cast<uint4*>(o + j * 16)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+            if (a.lse != nullptr && lo_half)
+                a.lse[g * kH + head] = (l_h > 0.f) ? (m_h + log2f(l_h)) / kLog2e : -INFINITY;
+        } else {
+            float* po = part_o + ((g * splits + sp) * kH + head) * kDv + dim0;
+            for (int j = 0; j < 256 / 16; ++j) {
+                uint32_t ov[16];
+                if (have) {
+                    tmem_ld16(tmem_addr(tmem, quarter * 32, j * 16), ov);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) ov[q] = 0;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    reinterpret_cast<uint4*>(po + j * 16)[q] = make_uint4(ov[4 * q], ov[4 * q + 1], ov[4 * q + 2], ov[4 * q + 3]);
+            }
+            if (lo_half) {
+                float* ml = part_ml + ((g * splits + sp) * kH + head) * 2;
+                ml[0] = (l_h > 0.f) ? m_h : -INFINITY;
+                ml[1] = l_h;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// Merges the split partials of each (query, head) in split order (fixed tree:
+// sequential), writing bf16 output and the natural-log LSE.
+__global__ void attend_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                                      int splits, void* __restrict__ out, float* __restrict__ lse) {
+    const int64_t gh = blockIdx.x;   // (query, head)
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[(gh / kH * splits + s) * kH * 2 + (gh % kH) * 2]);
+    float L = 0.f;
+    for (int s = 0; s < splits; ++s) {
+        const float* ml = part_ml + (gh / kH * splits + s) * kH * 2 + (gh % kH) * 2;
+        if (ml[1] > 0.f) L += ml[1] * exp2f(ml[0] - M);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int d = threadIdx.x; d < kDv; d += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float* ml = part_ml + (gh / kH * splits + s) * kH * 2 + (gh % kH) * 2;
+            if (ml[1] > 0.f)
+                acc += part_o[((gh / kH * splits + s) * kH + gh % kH) * kDv + d] * exp2f(ml[0] - M);
+        }
+        static_cast<uint16_t*>(out)[gh * kDv + d] = f32_to_bf16_bits(acc * inv);
+    }
+    if (lse != nullptr && threadIdx.x == 0) lse[gh] = L > 0.f ? (M + log2f(L)) / kLog2e : -INFINITY;
+}
+
+// --------------------------------------------------------------- fp32 path
+constexpr int kF32Chunk = 64;
+
+__global__ void attend_f32_kernel(const AttendArgs a, int* status) {
+    extern __shared__ float sh[];
+    const int H = a.H, D = a.D, dv = a.d_v;
+    float* qs = sh;                          // [H, D]
+    float* rows = qs + H * D;                // [chunk, D]
+    float* s = rows + kF32Chunk * D;         // [H, chunk]
+    float* o = s + H * kF32Chunk;            // [H, dv]
+    float* mh = o + H * dv;                  // [H]
+    float* lh = mh + H;                      // [H]
+    float* al = lh + H;                      // [H]
+    int* sel = reinterpret_cast<int*>(al + H);   // [k]
+    __shared__ int nsel_s;
+
+    const int64_t g = blockIdx.x, b = g / a.Q;
+    const float* qg = static_cast<const float*>(a.q) + g * H * D;
+    for (int i = threadIdx.x; i < H * D; i += blockDim.x) qs[i] = qg[i];
+    for (int i = threadIdx.x; i < H * dv; i += blockDim.x) o[i] = 0.f;
+    for (int i = threadIdx.x; i < H; i += blockDim.x) { mh[i] = -INFINITY; lh[i] = 0.f; }
+    if (threadIdx.x == 0) {
+        int n = 0;
+        if (a.idx != nullptr) {
+            for (int i = 0; i < a.k; ++i) {
+                int v = a.idx[g * a.k + i];
+                if (v >= a.N_c) { set_status(status, LCS_ERR_DEVICE, 202); v = -1; }
+                if (v >= 0) sel[n++] = v;
+            }
+        } else {
+            int64_t av = a.N_c;
+            if (a.q_pos != nullptr) {
+                av = (a.q_pos[g] + 1) / a.m;
+                av = av < 0 ? 0 : (av < a.N_c ? av : a.N_c);
+            }
+            n = (int)av;
+        }
+        nsel_s = n;
+    }
+    __syncthreads();
+    const RowPlan plan = plan_rows(a, g, nsel_s);
+    const int64_t R = plan.nsel + plan.nwin;
+    const int* selp = a.idx != nullptr ? sel : nullptr;
+    for (int64_t r0 = 0; r0 < R; r0 += kF32Chunk) {
+        const int nr = (int)((R - r0) < kF32Chunk ? (R - r0) : kF32Chunk);
+        for (int i = threadIdx.x; i < nr * D; i += blockDim.x) {
+            const int rr = i / D, c = i - rr * D;
+            rows[i] = reinterpret_cast<const float*>(row_ptr(a, b, plan, selp, r0 + rr, D * 4))[c];
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < H * nr; i += blockDim.x) {
+            const int h = i / nr, rr = i - h * nr;
+            float acc = 0.f;
+            for (int c = 0; c < D; ++c) acc = fmaf(qs[h * D + c], rows[rr * D + c], acc);
+            s[h * kF32Chunk + rr] = acc * a.scale;
+        }
+        __syncthreads();
+        for (int h = threadIdx.x; h < H; h += blockDim.x) {
+            float mx = mh[h];
+            for (int rr = 0; rr < nr; ++rr) mx = fmaxf(mx, s[h * kF32Chunk + rr]);
+            const float alpha = (mh[h] == -INFINITY) ? 0.f : expf(mh[h] - mx);
+            float l = lh[h] * alpha;
+            for (int rr = 0; rr < nr; ++rr) {
+                const float p = expf(s[h * kF32Chunk + rr] - mx);
+                s[h * kF32Chunk + rr] = p;
+                l += p;
+            }
+            mh[h] = mx;
+            lh[h] = l;
+            al[h] = alpha;
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < H * dv; i += blockDim.x) {
+            const int h = i / dv, c = i - h * dv;
+            float acc = o[i] * al[h];
+            for (int rr = 0; rr < nr; ++rr) acc = fmaf(s[h * kF32Chunk + rr], rows[rr * D + c], acc);
+            o[i] = acc;
+        }
+        __syncthreads();
+    }
+    float* og = static_cast<float*>(a.out) + g * H * dv;
+    for (int i = threadIdx.x; i < H * dv; i += blockDim.x) {
+        const int h = i / dv;
+        og[i] = lh[h] > 0.f ? o[i] / lh[h] : 0.f;
+    }
+    if (a.lse != nullptr)
+        for (int h = threadIdx.x; h < H; h += blockDim.x)
+            a.lse[g * H + h] = lh[h] > 0.f ? mh[h] + logf(lh[h]) : -INFINITY;
+}
+
+int choose_splits(const AttendArgs& a) {
+    const int64_t queries = a.B * a.Q;
+    const int64_t rmax = (a.idx != nullptr ? a.k : a.N_c) + (a.q_pos == nullptr ? a.Tw : (a.W < a.Tw ? a.W : a.Tw));
+    const int64_t chunks = (rmax + kChunk - 1) / kChunk;
+    int64_t s = num_sms() / (queries > 0 ? queries : 1);
+    if (s < 1) s = 1;
+    if (s > chunks) s = chunks > 0 ? chunks : 1;
+    // at least two chunks per split so the ring overlaps gather and math
+    while (s > 1 && (chunks + s - 1) / s < 2) --s;
+    return (int)s;
+}
+
+}  // namespace
+
+int64_t attend_scratch_bytes(const AttendArgs& a) {
+    if (a.kv_dtype == LCS_F32) return 0;
+    const int s = choose_splits(a);
+    if (s == 1) return 0;
+    const int64_t queries = a.B * a.Q;
+    return align256(queries * s * kH * kDv * 4) + align256(queries * s * kH * 2 * 4);
+}
+
+cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaStream_t s, bool pdl) {
+    const int64_t queries = a.B * a.Q;
+    if (queries == 0) return cudaSuccess;
+    if (a.kv_dtype == LCS_F32) {
+        const size_t smem = sizeof(float) * (a.H * a.D + kF32Chunk * a.D + a.H * kF32Chunk + a.H * a.d_v + 3 * a.H) +
+                            sizeof(int) * (a.k > 0 ? a.k : 1);
+        cudaError_t e = cudaFuncSetAttribute(attend_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_k(attend_f32_kernel, dim3((unsigned)queries), dim3(256), smem, s, pdl, a, status);
+    }
+    const int splits = choose_splits(a);
+    CUtensorMap mq;
+    if (!encode_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, kD, (uint64_t)(queries * kH), kD * 2, 64, kH,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    float* part_o = nullptr;
+    float* part_ml = nullptr;
+    if (splits > 1) {
+        part_o = static_cast<float*>(scratch);
+        part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256(queries * splits * kH * kDv * 4));
+    }
+    auto kern = (a.kv_dtype == LCS_KV_FP8) ? attend_tc_kernel<true> : attend_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
+    if (e != cudaSuccess) return e;
+    e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, a, splits, part_o,
+                 part_ml, status);
+    if (e != cudaSuccess || splits == 1) return e;
+    attend_combine_kernel<<<(unsigned)(queries * kH), 128, 0, s>>>(part_o, part_ml, splits, a.out, a.lse);
+    return cudaGetLastError();
+}
+
+}  // namespace lcs

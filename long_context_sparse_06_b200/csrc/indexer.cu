@@ -1,0 +1,271 @@
+// indexer.cu -- lightning-indexer scoring.
+//
+// "DeepSeek V4 深度解析" §2, CSA step 2: a light, low-rank indexer scores every
+// compressed entry against the query; "V3 vs V4" page, "V4 改进一" (闪电索引器).
+// Adopted form (the pages print none):
+//   score[s] = sum_{h < H_I} w_h * ReLU(qI_h . kI_s)
+// with the per-head dot in fp32 and the head sum as a fixed-order fma chain
+// (h = 0, 1, ...), so that the score of an entry does not depend on where it
+// sits in the batch or in the tile.
+//
+// Two paths:
+//  * fp32 inputs: CUDA cores, the dot itself a fixed-order fma chain over d.
+//  * bf16 inputs: tcgen05 tensor cores.  A CTA is persistent over (query group,
+//    128-key tile) work items.  Warp 0 streams key tiles [128 x 128] with TMA
+//    (128-byte swizzle) through a 4-stage ring and the group's query heads
+//    [64 x 128] into one of two slots; warp 1 issues tcgen05.mma (M = 128 keys,
+//    N = 64 heads, K = 128) into one of four TMEM accumulators; warps 2-5 read
+//    the accumulator rows (one key per thread) with tcgen05.ld and apply the
+//    ReLU / weighted head sum in fp32, writing one score per key.
+#include <utility>
+
+#include "lcs_common.cuh"
+#include "lcs_internal.h"
+
+namespace lcs {
+
+namespace {
+
+__device__ __forceinline__ int64_t avail(const int64_t* q_pos, int64_t g, int m, int64_t N_c) {
+    if (q_pos == nullptr) return N_c;
+    const int64_t a = (q_pos[g] + 1) / m;
+    return a < 0 ? 0 : (a < N_c ? a : N_c);
+}
+
+// ------------------------------------------------------------------ fp32 path
+__global__ void index_f32_kernel(const float* __restrict__ qI, const float* __restrict__ w,
+                                 const float* __restrict__ kI, int64_t Q, int64_t N_c, int H, int dI,
+                                 const int64_t* __restrict__ q_pos, int m, float* __restrict__ scores) {
+    extern __shared__ float sh[];
+    float* qs = sh;            // [H, dI]
+    float* ws = sh + H * dI;   // [H]
+    const int64_t g = blockIdx.x;   // (b, q)
+    const int64_t b = g / Q;
+    for (int i = threadIdx.x; i < H * dI; i += blockDim.x) qs[i] = qI[g * H * dI + i];
+    for (int i = threadIdx.x; i < H; i += blockDim.x) ws[i] = w[g * H + i];
+    __syncthreads();
+    const int64_t n = avail(q_pos, g, m, N_c);
+    const float* kb = kI + b * N_c * dI;
+    for (int64_t s = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; s < N_c; s += (int64_t)gridDim.y * blockDim.x) {
+        float acc = -INFINITY;
+        if (s < n) {
+            acc = 0.f;
+            const float* kr = kb + s * dI;
+            for (int h = 0; h < H; ++h) {
+                float dot = 0.f;
+                for (int c = 0; c < dI; ++c) dot = fmaf(qs[h * dI + c], kr[c], dot);
+                const float r = dot > 0.f ? dot : 0.f;
+                acc = fmaf(ws[h], r, acc);
+            }
+        }
+        scores[g * N_c + s] = acc;
+    }
+}
+
+// ------------------------------------------------------------- bf16 tcgen05 path
+constexpr int kBM = 128;        // keys per tile (MMA M)
+constexpr int kHeads = 64;      // index heads (MMA N)
+constexpr int kDI = 128;        // index dim (MMA K)
+constexpr int kStages = 4;
+constexpr int kAcc = 4;
+constexpr int kATile = kBM * kDI * 2;        // 32 KB
+constexpr int kBTile = kHeads * kDI * 2;     // 16 KB
+constexpr int kTmemCols = kAcc * kHeads;     // 256
+constexpr int kIxThreads = 192;
+constexpr size_t kIxSmem = 1024 + kStages * kATile + 2 * kBTile;
+
+struct IxBars {
+    uint64_t full[kStages], empty[kStages];
+    uint64_t bfull[2], bempty[2];
+    uint64_t afull[kAcc], aempty[kAcc];
+    uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(kIxThreads, 1)
+    index_bf16_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                         const float* __restrict__ w, int64_t Q, int64_t N_c, const int64_t* __restrict__ q_pos,
+                         int m, int64_t groups, float* __restrict__ scores, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ IxBars bars;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* a_tiles = smem;
+    uint8_t* b_tiles = smem + kStages * kATile;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tiles_per = (N_c + kBM - 1) / kBM;
+    const int64_t total = groups * tiles_per;
+    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+    const int64_t it0 = (int64_t)blockIdx.x * per;
+    const int64_t it1 = (it0 + per < total) ? it0 + per : total;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) { mbar_init(&bars.full[i], 1); mbar_init(&bars.empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&bars.bfull[i], 1); mbar_init(&bars.bempty[i], 1); }
+        for (int i = 0; i < kAcc; ++i) { mbar_init(&bars.afull[i], 1); mbar_init(&bars.aempty[i], 4); }
+        fence_barrier_init();
+        prefetch_tmap(&map_k);
+        prefetch_tmap(&map_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+
+#if defined(__CUDA_ARCH__)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int64_t prev_g = -1, gseq = -1, n_it = 0;
+            for (int64_t it = it0; it < it1; ++it) {
+                const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+                if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
+                if (g != prev_g) {
+                    ++gseq;
+                    const int slot = (int)(gseq & 1);
+                    if (!mbar_wait(&bars.bempty[slot], (uint32_t)(((gseq >> 1) & 1) ^ 1), status, 101)) break;
+                    mbar_arrive_expect_tx(&bars.bfull[slot], kBTile);
+                    for (int kb = 0; kb < 2; ++kb)
+                        tma_load_2d(b_tiles + slot * kBTile + kb * (kBTile / 2), &map_q, &bars.bfull[slot], kb * 64,
+                                    (int)(g * kHeads));
+                    prev_g = g;
+                }
+                const int st = (int)(n_it % kStages);
+                if (!mbar_wait(&bars.empty[st], (uint32_t)(((n_it / kStages) & 1) ^ 1), status, 102)) break;
+                mbar_arrive_expect_tx(&bars.full[st], kATile);
+                const int64_t b = g / Q;
+                for (int kb = 0; kb < 2; ++kb)
+                    tma_load_2d(a_tiles + st * kATile + kb * (kATile / 2), &map_k, &bars.full[st], kb * 64,
+                                (int)(b * N_c + tile * kBM));
+                ++n_it;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            constexpr uint32_t idesc = idesc_bf16(kBM, kHeads, false, false);
+            int64_t prev_g = -1, gseq = -1, n_it = 0;
+            int slot = 0;
+            bool ok = true;
+            for (int64_t it = it0; it < it1 && ok; ++it) {
+                const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+                if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
+                if (g != prev_g) {
+                    if (prev_g >= 0) mma_commit(&bars.bempty[slot]);   // previous group's heads are free
+                    ++gseq;
+                    slot = (int)(gseq & 1);
+                    if (!mbar_wait(&bars.bfull[slot], (uint32_t)((gseq >> 1) & 1), status, 103)) { ok = false; break; }
+                    prev_g = g;
+                }
+                const int st = (int)(n_it % kStages);
+                const int ac = (int)(n_it % kAcc);
+                if (!mbar_wait(&bars.aempty[ac], (uint32_t)(((n_it / kAcc) & 1) ^ 1), status, 104)) { ok = false; break; }
+                if (!mbar_wait(&bars.full[st], (uint32_t)((n_it / kStages) & 1), status, 105)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(a_tiles + st * kATile);
+                const uint32_t b_base = smem_u32(b_tiles + slot * kBTile);
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = sw128_desc(a_base + kb * (kATile / 2) + kk * 32, 16, 1024);
+                        const uint64_t bd = sw128_desc(b_base + kb * (kBTile / 2) + kk * 32, 16, 1024);
+                        mma_bf16_ss(tmem + ac * kHeads, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+                    }
+                mma_commit(&bars.empty[st]);
+                mma_commit(&bars.afull[ac]);
+                ++n_it;
+            }
+            if (prev_g >= 0) mma_commit(&bars.bempty[slot]);
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        int64_t prev_g = -1, n_it = 0;
+        float wr[kHeads];
+        for (int64_t it = it0; it < it1; ++it) {
+            const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+            const int64_t n = avail(q_pos, g, m, N_c);
+            if (tile * kBM >= n) continue;
+            if (g != prev_g) {
+#pragma unroll
+                for (int h = 0; h < kHeads; ++h) wr[h] = __ldg(w + g * kHeads + h);
+                prev_g = g;
+            }
+            const int ac = (int)(n_it % kAcc);
+            if (!mbar_wait(&bars.afull[ac], (uint32_t)((n_it / kAcc) & 1), status, 106)) break;
+            tc_fence_after();
+            uint32_t d[kHeads];
+#pragma unroll
+            for (int c = 0; c < kHeads / 16; ++c)
+                tmem_ld16(tmem_addr(tmem, quarter * 32, ac * kHeads + c * 16), *reinterpret_cast<uint32_t(*)[16]>(&d[c * 16]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.aempty[ac]);
+            float acc = 0.f;
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h) {
+                const float dot = __uint_as_float(d[h]);
+                acc = fmaf(wr[h], dot > 0.f ? dot : 0.f, acc);
+            }
+            const int64_t s = tile * kBM + row;
+            if (s < N_c) scores[g * N_c + s] = (s < n) ? acc : -INFINITY;
+            ++n_it;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_index_f32(const float* qI, const float* w, const float* kI, int64_t B, int64_t Q, int64_t N_c,
+                             int H_I, int d_I, const int64_t* q_pos, int m, float* scores, cudaStream_t s) {
+    const int64_t groups = B * Q;
+    if (groups == 0 || N_c == 0) return cudaSuccess;
+    const size_t smem = sizeof(float) * (H_I * d_I + H_I);
+    cudaError_t e = cudaFuncSetAttribute(index_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t ychunks = (N_c + 255) / 256;
+    dim3 grid((unsigned)groups, (unsigned)(ychunks < 16 ? ychunks : 16));
+    index_f32_kernel<<<grid, 256, smem, s>>>(qI, w, kI, Q, N_c, H_I, d_I, q_pos, m, scores);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_index_bf16_tc(const void* qI, const float* w, const void* kI, int64_t B, int64_t Q,
+                                 int64_t N_c, int d_I, const int64_t* q_pos, int m, float* scores, int* status,
+                                 cudaStream_t s, bool pdl) {
+    const int64_t groups = B * Q;
+    if (groups == 0 || N_c == 0) return cudaSuccess;
+    (void)d_I;
+    CUtensorMap mk, mq;
+    if (!encode_tmap_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kI, kDI, (uint64_t)(B * N_c), kDI * 2, 64, kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!encode_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qI, kDI, (uint64_t)(groups * kHeads), kDI * 2, 64,
+                        kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    cudaError_t e =
+        cudaFuncSetAttribute(index_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIxSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t total = groups * ((N_c + kBM - 1) / kBM);
+    const int64_t grid = total < num_sms() ? total : num_sms();
+    return launch_k(index_bf16_tc_kernel, dim3((unsigned)grid), dim3(kIxThreads), kIxSmem, s, pdl, mk, mq, w, Q, N_c,
+                    q_pos, m, groups, scores, status);
+}
+
+}  // namespace lcs

@@ -1,0 +1,89 @@
+// lcs_internal.h -- host-side launchers shared between the kernel files and the
+// C-ABI layer.  Launchers assume validated arguments and return a cudaError_t.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lcs {
+
+// Workspace layout: [0, 256) status word; then the op's scratch regions, each
+// 256-byte aligned.
+constexpr int64_t kStatusBytes = 256;
+inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+int num_sms();
+
+// compress.cu
+cudaError_t launch_compress(const void* x, int x_dtype, int64_t B, int64_t T, int d, const void* x_tail,
+                            const float* z_tail, const float* z, const float* bias, int m, int overlap, int d_rope,
+                            float theta, int64_t pos0, void* out, int out_dtype, cudaStream_t s);
+
+// misc.cu
+cudaError_t launch_rope(void* rows, int dtype, int64_t n, int d, int d_rope, float theta, const int64_t* pos,
+                        cudaStream_t s);
+cudaError_t launch_quant_kv_fp8(const float* x, int64_t n, int d_c, int d_r, void* out, cudaStream_t s);
+cudaError_t launch_quant_fp4(const float* x, int64_t n, int d, void* out, cudaStream_t s);
+cudaError_t launch_group_oproj(const float* o, int64_t T, int H, int d_v, const float* Wg, int G, int d_g,
+                               const float* Wo, int hidden, float* y, cudaStream_t s);
+
+// indexer.cu -- scores [B, Q, N_c] (fp32 or bf16)
+cudaError_t launch_index_f32(const float* qI, const float* w, const float* kI, int64_t B, int64_t Q, int64_t N_c,
+                             int H_I, int d_I, const int64_t* q_pos, int m, float* scores, cudaStream_t s);
+cudaError_t launch_index_bf16_tc(const void* qI, const float* w, const void* kI, int64_t B, int64_t Q,
+                                 int64_t N_c, int d_I, const int64_t* q_pos, int m, float* scores, int* status,
+                                 cudaStream_t s, bool pdl);
+cudaError_t launch_index_fp4_tc(const void* qI, const float* w, const void* kI, int64_t B, int64_t Q,
+                                int64_t N_c, int d_I, const int64_t* q_pos, int m, uint16_t* scores,
+                                uint8_t* q_scratch, int* status, cudaStream_t s, bool pdl);
+int64_t index_fp4_scratch_bytes(int64_t B, int64_t Q, int d_I);
+
+// topk.cu
+int64_t topk_scratch_bytes(int64_t rows, int64_t N_c);
+cudaError_t launch_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, int64_t N_c,
+                        const int64_t* q_pos, int m, int k, int32_t* idx, void* scratch, int* status,
+                        cudaStream_t s, bool pdl);
+
+// attend.cu
+struct AttendArgs {
+    const void* q;
+    const void* comp;
+    const void* win;
+    int kv_dtype;
+    int64_t B, Q, N_c, Tw;
+    const int32_t* idx;   // CSA selection or nullptr (HCA)
+    int k;
+    const int64_t* q_pos;
+    const int64_t* win_pos0;
+    int m;   // HCA availability stride
+    int W, H, D, d_v;
+    float scale;
+    void* out;
+    float* lse;
+};
+int64_t attend_scratch_bytes(const AttendArgs& a);
+cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaStream_t s, bool pdl);
+
+// Launch helper with optional programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                     Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+}  // namespace lcs

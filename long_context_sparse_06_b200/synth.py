@@ -80,3 +80,67 @@ def bf16_tensor(x):
     """Round float values to bf16 (torch's RNE conversion) -> torch CPU bf16 tensor."""
     import torch
     return torch.from_numpy(f32(x)).to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------
+# The same generator written with torch int64 ops, for large tensors generated
+# directly on a device.  Multiplication wraps modulo 2^64 and right shifts are
+# made logical with a mask, so the 64-bit stream is identical to the numpy one;
+# the Box-Muller doubles may differ from numpy's libm in the last ulp.
+def _u64_to_i64(v: int) -> int:
+    return v - (1 << 64) if v >= (1 << 63) else v
+
+
+_GAMMA_I = _u64_to_i64(0x9E3779B97F4A7C15)
+_M1_I = _u64_to_i64(0xBF58476D1CE4E5B9)
+_M2_I = _u64_to_i64(0x94D049BB133111EB)
+
+
+def _lsr_t(z, s: int):
+    return (z >> s) & ((1 << (64 - s)) - 1)
+
+
+def _mix_t(z):
+    z = (z ^ _lsr_t(z, 30)) * _M1_I
+    z = (z ^ _lsr_t(z, 27)) * _M2_I
+    return z ^ _lsr_t(z, 31)
+
+
+def uniform_t(name: str, n: int, seed: int = 0, device="cpu"):
+    import torch
+    key = _u64_to_i64(int(_key(name, seed)))
+    out = torch.empty(n, dtype=torch.float64, device=device)
+    for s in range(0, n, _CHUNK * 16):
+        e = min(n, s + _CHUNK * 16)
+        ctr = torch.arange(s + 1, e + 1, dtype=torch.int64, device=device)
+        x = _mix_t(ctr * _GAMMA_I + key)
+        out[s:e] = (_lsr_t(x, 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    return out
+
+
+def normal_t(name: str, shape, seed: int = 0, std: float = 1.0, dtype=None, device="cpu"):
+    """torch twin of normal(): N(0, std^2) of the given shape, cast to dtype."""
+    import torch
+    shape = tuple(shape) if np.iterable(shape) else (int(shape),)
+    n = int(np.prod(shape))
+    m = (n + 1) // 2
+    dtype = dtype or torch.float32
+    out = torch.empty(n, dtype=dtype, device=device)
+    step = _CHUNK * 8
+    key = _u64_to_i64(int(_key(name, seed)))
+    for s in range(0, m, step):
+        e = min(m, s + step)
+        ctr = torch.arange(2 * s + 1, 2 * e + 1, dtype=torch.int64, device=device)
+        u = (_lsr_t(_mix_t(ctr * _GAMMA_I + key), 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+        u1, u2 = u[0::2], u[1::2]
+        r = torch.sqrt(-2.0 * torch.log(u1))
+        z = torch.stack([r * torch.cos(2.0 * np.pi * u2), r * torch.sin(2.0 * np.pi * u2)], dim=1).reshape(-1)
+        lo, hi = 2 * s, min(n, 2 * e)
+        out[lo:hi] = (z[:hi - lo] * std).to(dtype)
+    return out.reshape(shape)
+
+
+def with_outliers_t(name: str, x, frac: float = 0.01, factor: float = 20.0, seed: int = 0):
+    import torch
+    u = uniform_t(name + ".outlier", x.numel(), seed, device=x.device).reshape(x.shape)
+    return torch.where(u < frac, x * factor, x)

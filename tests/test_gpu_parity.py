@@ -1,0 +1,384 @@
+"""GPU parity: every kernel of the hot path against the CPU oracle on seeded inputs.
+
+Sizes are small enough for the oracle to finish in seconds while spanning several
+tiles and a ragged tail.  Tolerances: integer / byte / index work bit-exact;
+fp32 outputs max-abs 1e-4; bf16 / FP8 outputs max-abs 2e-2 x RMS(oracle).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close_abs, assert_close_rel_rms, randn, topk_gap_ok
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import long_context_sparse_06_b200 as lcs
+    lcs.lib()
+    return lcs
+
+
+# ------------------------------------------------------------- codecs / RoPE
+def test_quant_kv_fp8_bit_exact(L, orc):
+    from long_context_sparse_06_b200 import synth
+    x = synth.with_outliers("g.kv8", synth.normal("g.kv8", (777, 576))).astype(np.float32)
+    gpu = L.lcs_quant_kv_fp8(torch.from_numpy(x).to(DEV)).cpu().numpy()
+    np.testing.assert_array_equal(gpu, orc.quant_kv_fp8(x))
+
+
+def test_quant_fp4_bit_exact(L, orc):
+    from long_context_sparse_06_b200 import synth
+    x = synth.with_outliers("g.fp4", synth.normal("g.fp4", (513, 128))).astype(np.float32)
+    x[5] = 0.0                                   # an all-zero vector: scale 1
+    x[6, :32] = 1e-9                             # a block whose amax/6 underflows E4M3
+    gpu = L.lcs_quant_fp4(torch.from_numpy(x).to(DEV)).cpu().numpy()
+    p, s = orc.quant_fp4(x)
+    np.testing.assert_array_equal(gpu[:513 * 64].reshape(513, 64), p)
+    np.testing.assert_array_equal(gpu[513 * 64:].reshape(513, 4), s)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_rope(L, orc, dtype):
+    x = randn("g.rope", (300, 64), dtype=dtype)
+    pos = torch.arange(300, dtype=torch.int64) * 3497 + 11
+    g = L.lcs_rope(x.to(DEV).clone(), pos.to(DEV), 16).float().cpu().numpy()
+    ref = orc.rope(x.double().numpy(), pos.numpy(), 16)
+    if dtype == torch.float32:
+        assert_close_abs(g, ref, 1e-5, "rope fp32")
+    else:
+        assert_close_rel_rms(g, ref, 1e-2, "rope bf16")
+
+
+# ------------------------------------------------------------------ compress
+@pytest.mark.parametrize("case", ["c1_f32", "csa_bf16_tail", "hca_bf16", "m1_identity"])
+def test_compress(L, orc, case):
+    if case == "c1_f32":
+        B, T, d, m, ov, dr, dt, pos0 = 2, 1024, 64, 4, 2, 16, torch.float32, 0
+    elif case == "csa_bf16_tail":
+        B, T, d, m, ov, dr, dt, pos0 = 2, 260, 576, 4, 2, 64, torch.bfloat16, 131072
+    elif case == "hca_bf16":
+        B, T, d, m, ov, dr, dt, pos0 = 2, 128 * 5, 576, 128, 0, 64, torch.bfloat16, 0
+    else:
+        B, T, d, m, ov, dr, dt, pos0 = 1, 96, 64, 1, 0, 0, torch.float32, 0
+    x = randn(f"g.cx.{case}", (B, T, d), dtype=dt)
+    z = randn(f"g.cz.{case}", (B, T))
+    bias = randn(f"g.cb.{case}", (m + ov,))
+    tail = zt = None
+    if case == "csa_bf16_tail":
+        tail = randn("g.ct", (B, ov, d), dtype=dt)
+        zt = randn("g.czt", (B, ov))
+    if m == 128:
+        out = L.hca_compress(x.to(DEV), z.to(DEV), bias.to(DEV), m=m, d_rope=dr, pos0=pos0)
+    else:
+        out = L.csa_compress(x.to(DEV), z.to(DEV), bias.to(DEV), m=m, overlap=ov, d_rope=dr, pos0=pos0,
+                             x_tail=None if tail is None else tail.to(DEV), z_tail=None if zt is None else zt.to(DEV))
+    g = out.float().cpu().numpy()
+    for b in range(B):
+        ref, _ = orc.compress(x[b].double().numpy(), z[b].double().numpy(), bias.double().numpy(), m, ov,
+                              d_rope=dr, pos0=pos0,
+                              x_tail=None if tail is None else tail[b].double().numpy(),
+                              z_tail=None if zt is None else zt[b].double().numpy())
+        if case == "m1_identity":
+            np.testing.assert_array_equal(g[b], x[b].numpy())
+        elif dt == torch.float32:
+            assert_close_abs(g[b], ref, 1e-4, case)
+        else:
+            assert_close_rel_rms(g[b], ref, 2e-2, case)
+
+
+# --------------------------------------------------------------------- top-k
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_topk_bit_exact_on_same_scores(L, orc, dtype):
+    rows, N = 7, 5000
+    s = randn("g.tk", (1, rows, N), std=4.0)
+    s[0, 1] = torch.round(s[0, 1])                 # heavy ties
+    s[0, 2] = 0.0
+    s[0, 2, ::7] = -0.0                            # signed zeros tie with +0
+    s[0, 3, 100:] = -1e30                          # almost all equal below the top
+    s = s.to(dtype)
+    for k in (1, 64, 512, 1024, 4999, 5000, 6000):
+        idx = L.lcs_topk(s.to(DEV), k).cpu().numpy()
+        for r in range(rows):
+            ref = orc.topk(s[0, r].float().numpy(), k)
+            np.testing.assert_array_equal(idx[0, r], ref, err_msg=f"row {r} k {k}")
+
+
+def test_topk_large_rows_and_causal(L, orc):
+    # rows longer than the shared-memory cache; causal availability per query
+    s = randn("g.tkl", (1, 3, 70000), std=3.0)
+    s[0, 1] = torch.round(s[0, 1] * 4) / 4
+    idx = L.lcs_topk(s.to(DEV), 1024).cpu().numpy()
+    for r in range(3):
+        np.testing.assert_array_equal(idx[0, r], orc.topk(s[0, r].numpy(), 1024))
+    q_pos = torch.tensor([[0, 3, 4, 100, 4095, 20000]], dtype=torch.int64)
+    s2 = randn("g.tkc", (1, 6, 5000))
+    idx = L.lcs_topk(s2.to(DEV), 64, q_pos=q_pos.to(DEV), m=4).cpu().numpy()
+    for r in range(6):
+        n = orc.n_avail(int(q_pos[0, r]), 4, 5000)
+        np.testing.assert_array_equal(idx[0, r], orc.topk(s2[0, r, :n].numpy(), 64))
+
+
+# ------------------------------------------------------------------- indexer
+def test_index_f32_bit_exact(L, orc):
+    """C1 indexer shape: 4 heads x 32 dims, causal over 256 entries."""
+    B, Q, H, dI, Nc, k = 1, 200, 4, 32, 256, 64
+    qI = randn("g.i32.q", (B, Q, H, dI))
+    w = randn("g.i32.w", (B, Q, H), std=0.5)
+    kI = randn("g.i32.k", (B, Nc, dI))
+    q_pos = (torch.arange(Q, dtype=torch.int64) * 5 + 3).reshape(B, Q)
+    idx, sc = L.csa_index_topk(qI.to(DEV), w.to(DEV), kI.to(DEV), k, q_pos=q_pos.to(DEV), m=4, want_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    for q in range(Q):
+        n = orc.n_avail(int(q_pos[0, q]), 4, Nc)
+        ref = orc.index_scores_f32(qI[0, q].numpy(), w[0, q].numpy(), kI[0, :n].numpy())
+        np.testing.assert_array_equal(sc[0, q, :n], ref)
+        np.testing.assert_array_equal(idx[0, q], orc.topk(ref, k))
+
+
+def _bf16_score_bound(qI, w, kI):
+    """|GPU - oracle| bound for bf16 scores: each per-head dot from the tensor
+    cores carries at most (d_I/16 + 1) fp32 roundings (or truncations) of partial
+    sums bounded by sum|q||k|; the head chain adds H roundings."""
+    qa, ka = np.abs(qI), np.abs(kI)
+    sabs = ka @ qa.T                                   # [N, H]
+    dI = qI.shape[1]
+    dot_err = (dI // 16 + 1) * 2.0 ** -23 * sabs
+    relu_abs = sabs                                    # |relu(dot)| <= sum|q||k|
+    return dot_err @ np.abs(w) * 1.01 + relu_abs @ np.abs(w) * (w.size + 2) * 2.0 ** -24
+
+
+def test_index_bf16_tensor_cores(L, orc):
+    B, H, dI, Nc, k = 6, 64, 128, 1500, 128           # 12 tiles per request, ragged last tile
+    qI = randn("g.ib.q", (B, 1, H, dI), dtype=torch.bfloat16)
+    w = randn("g.ib.w", (B, 1, H), std=1 / 8)
+    kI = randn("g.ib.k", (B, Nc, dI), dtype=torch.bfloat16)
+    idx, sc = L.csa_index_topk(qI.to(DEV), w.to(DEV), kI.to(DEV), k, want_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    exact_rows = 0
+    for b in range(B):
+        qd, kd, wd = qI[b, 0].double().numpy(), kI[b].double().numpy(), w[b, 0].numpy()
+        ref = orc.index_scores_bf16(qd, wd, kd)
+        bound = _bf16_score_bound(qd, wd, kd)
+        err = np.abs(sc[b, 0].astype(np.float64) - ref)
+        assert np.all(err <= bound), f"b={b}: max err/bound {np.max(err / bound):.3f}"
+        # level 1: the selection on the GPU's own scores is the oracle's selection
+        np.testing.assert_array_equal(idx[b, 0], orc.topk(sc[b, 0], k))
+        # level 3: when the oracle's k-th gap exceeds twice the bound, the sets agree
+        if topk_gap_ok(ref, k, bound.max()):
+            np.testing.assert_array_equal(idx[b, 0], orc.topk(ref, k))
+            exact_rows += 1
+    assert exact_rows >= B // 2
+
+
+def test_index_bf16_causal_prefill(L, orc):
+    B, Q, H, dI, Nc, k = 1, 40, 64, 128, 700, 64
+    qI = randn("g.ic.q", (B, Q, H, dI), dtype=torch.bfloat16)
+    w = randn("g.ic.w", (B, Q, H), std=1 / 8)
+    kI = randn("g.ic.k", (B, Nc, dI), dtype=torch.bfloat16)
+    q_pos = (torch.arange(Q, dtype=torch.int64) * 71 + 2).reshape(B, Q)
+    idx, sc = L.csa_index_topk(qI.to(DEV), w.to(DEV), kI.to(DEV), k, q_pos=q_pos.to(DEV), m=4, want_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    for q in range(Q):
+        n = orc.n_avail(int(q_pos[0, q]), 4, Nc)
+        qd, kd, wd = qI[0, q].double().numpy(), kI[0, :n].double().numpy(), w[0, q].numpy()
+        ref = orc.index_scores_bf16(qd, wd, kd)
+        if n:
+            assert np.all(np.abs(sc[0, q, :n] - ref) <= _bf16_score_bound(qd, wd, kd))
+        np.testing.assert_array_equal(idx[0, q], orc.topk(sc[0, q, :n], k))
+
+
+# ----------------------------------------------------------------- attention
+def test_attend_f32_c1(L, orc):
+    """C1 attention shape: 8 heads, D = 64 (48 + 16), d_v = 48, k = 64, window 128, causal."""
+    B, Q, H, D, dv, Nc, k, W = 1, 160, 8, 64, 48, 256, 64, 128
+    T = 1024
+    q = randn("g.a32.q", (B, Q, H, D))
+    comp = randn("g.a32.c", (B, Nc, D))
+    win = randn("g.a32.w", (B, T, D))
+    q_pos = (torch.arange(Q, dtype=torch.int64) * 6 + 5).reshape(B, Q)
+    rng = np.random.default_rng(0)
+    idx = np.full((B, Q, k), -1, np.int32)
+    for q_ in range(Q):
+        n = orc.n_avail(int(q_pos[0, q_]), 4, Nc)
+        take = min(k, n)
+        if take:
+            idx[0, q_, :take] = np.sort(rng.choice(n, take, replace=False))
+    wp0 = torch.zeros(B, dtype=torch.int64)
+    out, lse = L.csa_attend(q.to(DEV), comp.to(DEV), win.to(DEV), torch.from_numpy(idx).to(DEV), dv, 1 / 8,
+                            q_pos=q_pos.to(DEV), win_pos0=wp0.to(DEV), W=W, want_lse=True)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for q_ in range(Q):
+        o, l = orc.csa_attend(q[0, q_].double().numpy(), comp[0].double().numpy(), idx[0, q_],
+                              win[0].double().numpy(), 0, int(q_pos[0, q_]), W, dv, 1 / 8)
+        assert_close_abs(out[0, q_], o, 1e-4, f"q {q_}")
+        assert_close_abs(lse[0, q_], l, 1e-4, f"lse q {q_}")
+
+
+def _rand_sel(name, B, Q, k, navail):
+    rng = np.random.default_rng(abs(hash(name)) % 2 ** 32)
+    idx = np.full((B, Q, k), -1, np.int32)
+    for b in range(B):
+        for q in range(Q):
+            n = navail[b][q] if isinstance(navail, list) else navail
+            t = min(k, n)
+            if t:
+                idx[b, q, :t] = np.sort(rng.choice(n, t, replace=False))
+    return idx
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_csa_attend_decode_tc(L, orc, kv):
+    B, H, D, dv, Nc, k, Tw = 5, 64, 576, 512, 3000, 512, 128
+    scale = 1 / math.sqrt(576)
+    q = randn(f"g.ad.q.{kv}", (B, 1, H, D), dtype=torch.bfloat16)
+    comp32 = randn(f"g.ad.c.{kv}", (B, Nc, D))
+    win32 = randn(f"g.ad.w.{kv}", (B, Tw, D))
+    idx = _rand_sel(f"sel.{kv}", B, 1, k, Nc)
+    idx[1, 0, 300:] = -1                         # a short selection
+    idx[2, 0, :] = -1                            # window only
+    if kv == "bf16":
+        comp, win = comp32.to(torch.bfloat16), win32.to(torch.bfloat16)
+        comp_g, win_g, kvd = comp.to(DEV), win.to(DEV), L.BF16
+        comp_d, win_d = comp.double().numpy(), win.double().numpy()
+    else:
+        comp_g = L.lcs_quant_kv_fp8(comp32.to(DEV))
+        win_g = L.lcs_quant_kv_fp8(win32.to(DEV))
+        kvd = L.KV_FP8
+        comp_d = orc.dequant_kv_fp8(orc.quant_kv_fp8(comp32.numpy()))
+        win_d = orc.dequant_kv_fp8(orc.quant_kv_fp8(win32.numpy()))
+    out, lse = L.csa_attend(q.to(DEV), comp_g, win_g, torch.from_numpy(idx).to(DEV), dv, scale, kv_dtype=kvd,
+                            want_lse=True)
+    out, lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        o, l = orc.csa_attend(q[b, 0].double().numpy(), comp_d[b], idx[b, 0], win_d[b], 0, -1, 128, dv, scale)
+        assert_close_rel_rms(out[b, 0], o, 2e-2, f"{kv} b {b}")
+        assert_close_abs(lse[b, 0], l, 2e-2, f"{kv} lse b {b}")
+
+
+def test_hca_attend_decode_tc(L, orc):
+    B, H, D, dv, Nc, Tw = 3, 64, 576, 512, 1100, 128     # many chunks, several splits
+    scale = 1 / math.sqrt(576)
+    q = randn("g.h.q", (B, 1, H, D), dtype=torch.bfloat16)
+    comp = randn("g.h.c", (B, Nc, D), dtype=torch.bfloat16)
+    win = randn("g.h.w", (B, Tw, D), dtype=torch.bfloat16)
+    out, lse = L.hca_attend(q.to(DEV), comp.to(DEV), win.to(DEV), dv, scale, want_lse=True)
+    out, lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        o, l = orc.hca_attend(q[b, 0].double().numpy(), comp[b].double().numpy(), 128, win[b].double().numpy(), 0,
+                              -1, 128, dv, scale)
+        assert_close_rel_rms(out[b, 0], o, 2e-2, f"hca b {b}")
+        assert_close_abs(lse[b, 0], l, 2e-2, f"hca lse b {b}")
+
+
+def test_attend_prefill_tc_causal(L, orc):
+    """C4-shaped (smaller): queries at positions p0.., window from the chunk plus a 127-row prefix tail."""
+    B, Q, H, D, dv, k, W = 1, 24, 64, 576, 512, 256, 128
+    p0 = 4000
+    Nc = (p0 + Q) // 4
+    Tw = 127 + Q
+    scale = 1 / math.sqrt(576)
+    q = randn("g.ap.q", (B, Q, H, D), dtype=torch.bfloat16)
+    comp = randn("g.ap.c", (B, Nc, D), dtype=torch.bfloat16)
+    win = randn("g.ap.w", (B, Tw, D), dtype=torch.bfloat16)
+    q_pos = (p0 + torch.arange(Q, dtype=torch.int64)).reshape(B, Q)
+    wp0 = torch.tensor([p0 - 127], dtype=torch.int64)
+    nav = [[orc.n_avail(int(t), 4, Nc) for t in q_pos[0]]]
+    idx = _rand_sel("sel.pf", B, Q, k, nav)
+    out = L.csa_attend(q.to(DEV), comp.to(DEV), win.to(DEV), torch.from_numpy(idx).to(DEV), dv, scale,
+                       q_pos=q_pos.to(DEV), win_pos0=wp0.to(DEV)).float().cpu().numpy()
+    for t in range(Q):
+        o, _ = orc.csa_attend(q[0, t].double().numpy(), comp[0].double().numpy(), idx[0, t],
+                              win[0].double().numpy(), p0 - 127, int(q_pos[0, t]), W, dv, scale)
+        assert_close_rel_rms(out[0, t], o, 2e-2, f"prefill q {t}")
+    # HCA causal with m' = 128 on the same queries
+    Nh = (p0 + Q) // 128
+    outh = L.hca_attend(q.to(DEV), comp[:, :Nh].contiguous().to(DEV), win.to(DEV), dv, scale, q_pos=q_pos.to(DEV),
+                        win_pos0=wp0.to(DEV), m=128).float().cpu().numpy()
+    for t in range(0, Q, 5):
+        o, _ = orc.hca_attend(q[0, t].double().numpy(), comp[0, :Nh].double().numpy(), 128, win[0].double().numpy(),
+                              p0 - 127, int(q_pos[0, t]), W, dv, scale)
+        assert_close_rel_rms(outh[0, t], o, 2e-2, f"hca prefill q {t}")
+
+
+# -------------------------------------------------------------- fused decode
+def test_decode_fused_csa_bf16(L, orc):
+    B, H, D, dv, Nc, k, Tw, HI, dI = 4, 64, 576, 512, 2500, 256, 128, 64, 128
+    scale = 1 / math.sqrt(576)
+    q = randn("g.df.q", (B, H, D), dtype=torch.bfloat16)
+    comp = randn("g.df.c", (B, Nc, D), dtype=torch.bfloat16)
+    win = randn("g.df.w", (B, Tw, D), dtype=torch.bfloat16)
+    qI = randn("g.df.qi", (B, HI, dI), dtype=torch.bfloat16)
+    w = randn("g.df.wi", (B, HI), std=1 / 8)
+    kI = randn("g.df.ki", (B, Nc, dI), dtype=torch.bfloat16)
+    idx_out = torch.empty((B, k), dtype=torch.int32, device=DEV)
+    out = L.decode_fused(L.MODE_CSA, q.to(DEV), comp.to(DEV), win.to(DEV), dv, scale, qI=qI.to(DEV), w=w.to(DEV),
+                         kI=kI.to(DEV), k=k, idx_out=idx_out)
+    out, idx = out.float().cpu().numpy(), idx_out.cpu().numpy()
+    for b in range(B):
+        qd, kd, wd = qI[b].double().numpy(), kI[b].double().numpy(), w[b].numpy()
+        ref_s = orc.index_scores_bf16(qd, wd, kd)
+        if topk_gap_ok(ref_s, k, _bf16_score_bound(qd, wd, kd).max()):
+            np.testing.assert_array_equal(idx[b], orc.topk(ref_s, k))
+        o, _ = orc.csa_attend(q[b].double().numpy(), comp[b].double().numpy(), idx[b], win[b].double().numpy(), 0,
+                              -1, 128, dv, scale)
+        assert_close_rel_rms(out[b], o, 2e-2, f"fused b {b}")
+
+
+def test_decode_fused_hca(L, orc):
+    B, H, D, dv, Nc, Tw = 2, 64, 576, 512, 900, 128
+    scale = 1 / math.sqrt(576)
+    q = randn("g.dh.q", (B, H, D), dtype=torch.bfloat16)
+    comp = randn("g.dh.c", (B, Nc, D), dtype=torch.bfloat16)
+    win = randn("g.dh.w", (B, Tw, D), dtype=torch.bfloat16)
+    out = L.decode_fused(L.MODE_HCA, q.to(DEV), comp.to(DEV), win.to(DEV), dv, scale).float().cpu().numpy()
+    for b in range(B):
+        o, _ = orc.hca_attend(q[b].double().numpy(), comp[b].double().numpy(), 128, win[b].double().numpy(), 0, -1,
+                              128, dv, scale)
+        assert_close_rel_rms(out[b], o, 2e-2, f"fused hca b {b}")
+
+
+# --------------------------------------------------------- grouped projection
+def test_group_oproj(L, orc):
+    T, H, dv, G, dg, hidden = 300, 8, 48, 2, 64, 256
+    o = randn("g.gp.o", (T, H, dv))
+    Wg = randn("g.gp.g", (G, H // G * dv, dg), std=1 / math.sqrt(H // G * dv))
+    Wo = randn("g.gp.w", (G * dg, hidden), std=1 / math.sqrt(G * dg))
+    y = L.group_oproj(o.to(DEV), Wg.to(DEV), Wo.to(DEV)).cpu().numpy()
+    for t in range(0, T, 7):
+        assert_close_abs(y[t], orc.group_oproj(o[t].double().numpy(), Wg.double().numpy(), Wo.double().numpy()),
+                         1e-4, f"t {t}")
+
+
+# ------------------------------------------------- determinism and invariance
+def test_determinism_and_batch_invariance(L):
+    B, H, D, dv, Nc, k, Tw = 4, 64, 576, 512, 1800, 256, 128
+    scale = 1 / math.sqrt(576)
+    q = randn("g.di.q", (B, H, D), dtype=torch.bfloat16).to(DEV)
+    comp = randn("g.di.c", (B, Nc, D), dtype=torch.bfloat16).to(DEV)
+    win = randn("g.di.w", (B, Tw, D), dtype=torch.bfloat16).to(DEV)
+    qI = randn("g.di.qi", (B, 64, 128), dtype=torch.bfloat16).to(DEV)
+    w = randn("g.di.wi", (B, 64), std=1 / 8).to(DEV)
+    kI = randn("g.di.ki", (B, Nc, 128), dtype=torch.bfloat16).to(DEV)
+    args = dict(qI=qI, w=w, kI=kI, k=k)
+    o1 = L.decode_fused(L.MODE_CSA, q, comp, win, dv, scale, **args)
+    o2 = L.decode_fused(L.MODE_CSA, q, comp, win, dv, scale, **args)
+    assert torch.equal(o1, o2)
+    perm = torch.tensor([2, 0, 3, 1], device=DEV)
+    o3 = L.decode_fused(L.MODE_CSA, q[perm].contiguous(), comp[perm].contiguous(), win[perm].contiguous(), dv, scale,
+                        qI=qI[perm].contiguous(), w=w[perm].contiguous(), kI=kI[perm].contiguous(), k=k)
+    assert torch.equal(o3, o1[perm])
+    # the selection does not depend on the batch at all
+    i1 = torch.empty((B, k), dtype=torch.int32, device=DEV)
+    i4 = torch.empty((1, k), dtype=torch.int32, device=DEV)
+    L.decode_fused(L.MODE_CSA, q, comp, win, dv, scale, idx_out=i1, **args)
+    L.decode_fused(L.MODE_CSA, q[1:2].contiguous(), comp[1:2].contiguous(), win[1:2].contiguous(), dv, scale,
+                   qI=qI[1:2].contiguous(), w=w[1:2].contiguous(), kI=kI[1:2].contiguous(), k=k, idx_out=i4)
+    assert torch.equal(i4[0], i1[1])
