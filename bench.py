@@ -225,6 +225,9 @@ def run_gpu(args):
 
     # ---- per-stage device time of the same steps (events on the launching stream)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in evs:   # torch creates the CUDA event on its first record
+        e.record(stream)
+    torch.cuda.synchronize()
     handles = (lcs.C.c_void_p * 4)(*[e.cuda_event for e in evs])
     stage_ms = [0.0, 0.0, 0.0]
     lcs.lib().lcs_set_stage_events(handles, 4)

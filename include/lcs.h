@@ -163,7 +163,9 @@ LCS_API int lcs_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, 
  *   q    [B, Q, H, D]   LCS_F32 with kv LCS_F32; LCS_BF16 with kv LCS_BF16 or LCS_KV_FP8
  *   comp [B, N_c, row]  kv_dtype (row = D elements, or 656 bytes for LCS_KV_FP8)
  *   win  [B, Tw, row]   kv_dtype
- *   idx  [B, Q, k]      int32, -1 = unused slot
+ *   idx  [B, Q, k]      int32 selection: valid entries first, then -1 padding (the form
+ *                       csa_index_topk returns); the first -1 ends the selection.  An
+ *                       index >= N_c also ends it and records LCS_ERR_DEVICE.
  *   q_pos [B, Q], win_pos0 [B]  int64 device arrays, or both NULL (decode)
  *   out  [B, Q, H, d_v] out_dtype (LCS_F32 for f32 kv, LCS_BF16 otherwise)
  *   lse  [B, Q, H]      fp32 natural-log sum of exp(scale*q.K) over R, or NULL
@@ -228,8 +230,9 @@ LCS_API int lcs_rope(void* rows, int dtype, int64_t n, int d, int d_rope, float 
  * Cache writers for the two quantised formats ("DeepSeek V4 深度解析" §2 last
  * paragraph and §4).
  *   lcs_quant_kv_fp8: x [n, d_c + d_r] fp32 -> LCS_KV_FP8 rows [n, d_c + 2 d_r + 4 d_c/128]:
- *     per 128-block scale = amax/448 (fp32; 1 when amax is 0), code = E4M3(x/scale),
- *     round to nearest even, saturating; the d_r RoPE dims rounded to bf16.
+ *     per 128-block scale = the smallest power of two >= amax/448 (amax/448 in fp32;
+ *     1 when amax is 0), code = E4M3(x/scale), round to nearest even; the d_r RoPE
+ *     dims rounded to bf16.  The power-of-two scale makes code*scale exact in bf16.
  *   lcs_quant_fp4: x [n, d] fp32 -> LCS_FP4 planes (out: n*d/2 + n*d/32 bytes):
  *     per 32-block scale = E4M3(amax/6) (1 when that is 0), code = E2M1(x/scale).
  * d_c % 128 == 0, d % 32 == 0.

@@ -20,10 +20,12 @@
 //    cp.async (bf16) or load-convert-store (FP8 rows: E4M3 x block scale ->
 //    bf16), writing the SW128 layout that both MMAs read (the same bytes are
 //    the K-major B of Q.K^T and the MN-major B of P.V);
-//  * warps 0-3 run the online softmax on S (fp32, exp2), write P as bf16 into
-//    the chunk's RoPE column block (dead once Q.K^T has read it), rescale O in
-//    TMEM only when a head's running max grows by more than 2^8 in weight, and
-//    finally normalise O and write it out (or a split partial for the combine).
+//  * warps 0-3 run the online softmax on S (fp32, exp2) and write P as two bf16
+//    parts, P = P_hi + P_lo (P_hi into the chunk's RoPE column block, dead once
+//    Q.K^T has read it; P_lo into its own buffer), so P.V carries ~16 bits of P;
+//    they rescale O in TMEM only when a head's running max grows by more than
+//    2^8 in weight, and finally normalise O and write it out (or a split
+//    partial for the combine).
 // F32 path (C1-sized problems): CUDA cores, fp32 online softmax.
 #include <utility>
 
@@ -40,7 +42,7 @@ constexpr int kStageBytes = 9 * kBlk;         // 72 KB
 constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
 constexpr int kMaxK = 2048;
 constexpr int kAtThreads = 288;
-constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kMaxK * 4;
+constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kBlk;   // + the P_lo buffer
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
 
@@ -80,10 +82,11 @@ __device__ __forceinline__ RowPlan plan_rows(const AttendArgs& a, int64_t g, int
 }
 
 // Row pointer of row position r of query g (bf16 rows: D elements; FP8: 656 B).
+// sel = the query's selection (CSA; its first nsel entries are valid) or null (HCA).
 __device__ __forceinline__ const uint8_t* row_ptr(const AttendArgs& a, int64_t b, const RowPlan& p,
-                                                  const int* sel, int64_t r, int row_bytes) {
+                                                  const int32_t* sel, int64_t r, int row_bytes) {
     if (r < p.nsel) {
-        const int64_t e = sel ? sel[r] : r;
+        const int64_t e = sel ? __ldg(sel + r) : r;
         return static_cast<const uint8_t*>(a.comp) + (b * a.N_c + e) * row_bytes;
     }
     return static_cast<const uint8_t*>(a.win) + (b * a.Tw + p.win_lo + (r - p.nsel)) * row_bytes;
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* q_s = smem;
     uint8_t* stage_s = smem + kQBytes;
-    int* sel_s = reinterpret_cast<int*>(smem + kQBytes + 2 * kStageBytes);
+    uint8_t* plo_s = smem + kQBytes + 2 * kStageBytes;   // P_lo [64 heads x 64 rows] bf16, SW128
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g = blockIdx.x / splits;
@@ -125,21 +128,20 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 #if defined(__CUDA_ARCH__)
     asm volatile("griddepcontrol.wait;" ::: "memory");
 #endif
-    // ---- selection list (CSA: valid entries of idx in order; HCA: implicit)
+    // ---- selection length (CSA: the valid prefix of idx, as top-k emits it; HCA: n_avail).
+    // An index >= N_c ends the prefix and is reported through the status word.
     if (a.idx != nullptr) {
         if (warp == 0) {
             const int32_t* ir = a.idx + g * a.k;
-            int cnt = 0;
-            for (int base = 0; base < a.k; base += 32) {
+            int n = a.k;
+            for (int base = 0; base < a.k && n == a.k; base += 32) {
                 const int i = base + lane;
-                int32_t v = (i < a.k) ? ir[i] : -1;
-                if (v >= a.N_c) { set_status(status, LCS_ERR_DEVICE, 201); v = -1; }
-                const bool ok = v >= 0;
-                const uint32_t bal = __ballot_sync(0xffffffffu, ok);
-                if (ok) sel_s[cnt + __popc(bal & ((1u << lane) - 1u))] = v;
-                cnt += __popc(bal);
+                const int32_t v = (i < a.k) ? ir[i] : 0;
+                if (i < a.k && v >= a.N_c) set_status(status, LCS_ERR_DEVICE, 201);
+                const uint32_t bad = __ballot_sync(0xffffffffu, i < a.k && (v < 0 || v >= a.N_c));
+                if (bad) n = base + __ffs(bad) - 1;
             }
-            if (lane == 0) bars.nsel = cnt;
+            if (lane == 0) bars.nsel = n;
         }
     } else if (threadIdx.x == 0) {
         int64_t n = a.N_c;
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
-    const int* sel = (a.idx != nullptr) ? sel_s : nullptr;
+    const int32_t* sel = (a.idx != nullptr) ? a.idx + g * a.k : nullptr;
     const RowPlan plan = plan_rows(a, g, bars.nsel);
     const int64_t R = plan.nsel + plan.nwin;
     const int64_t nch_all = (R + kChunk - 1) / kChunk;
@@ -197,15 +199,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 const int st = c & 1;
                 if (!mbar_wait(&bars.pfull[st], (uint32_t)((c >> 1) & 1), status, 303)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t p_base = smem_u32(stage_s + st * kStageBytes + 8 * kBlk);
+                const uint32_t phi_base = smem_u32(stage_s + st * kStageBytes + 8 * kBlk);
+                const uint32_t plo_base = smem_u32(plo_s);
                 const uint32_t v_base = smem_u32(stage_s + st * kStageBytes);
 #pragma unroll
                 for (int half = 0; half < 2; ++half)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = sw128_desc(p_base + kk * 32, 16, 1024);
                         const uint64_t bd = sw128_desc(v_base + half * 4 * kBlk + kk * 2048, kBlk, 1024);
-                        mma_bf16_ss(tmem + (half ? (16u << 16) : 0u), ad, bd, idesc_pv, (c | kk) ? 1u : 0u);
+                        const uint32_t d_t = tmem + (half ? (16u << 16) : 0u);
+                        mma_bf16_ss(d_t, sw128_desc(phi_base + kk * 32, 16, 1024), bd, idesc_pv, (c | kk) ? 1u : 0u);
+                        mma_bf16_ss(d_t, sw128_desc(plo_base + kk * 32, 16, 1024), bd, idesc_pv, 1u);
                     }
                 mma_commit(&bars.kempty[st]);
                 mma_commit(&bars.ofull);
@@ -305,29 +309,21 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 rescale = (c > 0);
                 m_used = m_new;
             }
-            // P (bf16) for this thread's head into the chunk's RoPE block (K-major, 128 B per head row)
-            uint8_t* pblk = stage_s + st * kStageBytes + 8 * kBlk;
+            // P = exp2(scale*s*log2e - m) of this thread's head (lanes 0..15 own the heads)
             float psum = 0.f;
             if (lo_half) {
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int j0 = ch * 8 + 2 * q;
-                        float p0 = (j0 < nvalid) ? exp2f(__uint_as_float(sv[j0]) * sl2 - m_used) : 0.f;
-                        float p1 = (j0 + 1 < nvalid) ? exp2f(__uint_as_float(sv[j0 + 1]) * sl2 - m_used) : 0.f;
-                        pk[q] = pack_bf16x2(p0, p1);
-                        psum += bf16_bits_to_f32((uint16_t)(pk[q] & 0xFFFF)) + bf16_bits_to_f32((uint16_t)(pk[q] >> 16));
-                    }
-                    *reinterpret_cast<uint4*>(pblk + sw128_off(head, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                for (int j = 0; j < kChunk; ++j) {
+                    const float p = (j < nvalid) ? exp2f(__uint_as_float(sv[j]) * sl2 - m_used) : 0.f;
+                    sv[j] = __float_as_uint(p);
+                    psum += p;
                 }
             }
             l_sum = l_sum * alpha + psum;
+            // P_lo and O are shared with the previous chunk's P.V: wait until it is done
+            if (c > 0 && !mbar_wait(&bars.ofull, (uint32_t)((c - 1) & 1), status, 321)) break;
+            tc_fence_after();
             if (__any_sync(0xffffffffu, rescale)) {
-                // O must be stable: wait for the previous chunk's P.V
-                if (!mbar_wait(&bars.ofull, (uint32_t)((c - 1) & 1), status, 321)) break;
-                tc_fence_after();
                 const float f = rescale ? alpha : 1.f;
                 for (int j = 0; j < 256 / 16; ++j) {
                     uint32_t ov[16];
@@ -339,7 +335,26 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                     tmem_st16(ta, ov);
                 }
                 tmem_st_wait();
-                tc_fence_before();
+            }
+            tc_fence_before();
+            // P_hi = bf16(P) into the chunk's RoPE block, P_lo = bf16(P - P_hi) into its buffer
+            // (K-major SW128 rows of 128 B per head)
+            if (lo_half) {
+                uint8_t* phi = stage_s + st * kStageBytes + 8 * kBlk;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float p0 = __uint_as_float(sv[ch * 8 + 2 * q]);
+                        const float p1 = __uint_as_float(sv[ch * 8 + 2 * q + 1]);
+                        hi[q] = pack_bf16x2(p0, p1);
+                        lo[q] = pack_bf16x2(p0 - bf16_bits_to_f32((uint16_t)(hi[q] & 0xFFFF)),
+                                            p1 - bf16_bits_to_f32((uint16_t)(hi[q] >> 16)));
+                    }
+                    *reinterpret_cast<uint4*>(phi + sw128_off(head, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4*>(plo_s + sw128_off(head, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars.pfull[st]);

@@ -4,7 +4,8 @@
 //  * RoPE: rotate-half pairs on the last d_rope dims (the RoPE dims that
 //    "DeepSeek V4 深度解析" §2 keeps in BF16).
 //  * lcs_quant_kv_fp8: the mixed-precision KV row of the same paragraph (RoPE
-//    dims BF16, the rest FP8 E4M3 with one fp32 scale per 128 dims).
+//    dims BF16, the rest FP8 E4M3 with one power-of-two fp32 scale per 128
+//    dims, so that code * scale is exact in bf16).
 //  * lcs_quant_fp4: FP4 E2M1 with one E4M3 scale per 32 elements, the format of
 //    the indexer's QK path ("DeepSeek V4 深度解析" §4, FP4量化感知訓練).
 //  * group_oproj: the grouped output projection (§2, HCA paragraph).
@@ -58,8 +59,10 @@ __global__ void quant_kv_fp8_kernel(const float* __restrict__ x, int64_t n, int 
         const float4 v = *reinterpret_cast<const float4*>(xr + b * 128 + 4 * lane);
         float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
         amax = warp_max(amax);
-        float sc = amax / 448.0f;
-        if (sc == 0.0f) sc = 1.0f;
+        // smallest power of two >= amax/448: round the fp32 bit pattern up to the next exponent
+        const float t = amax / 448.0f;
+        const uint32_t tb = __float_as_uint(t);
+        const float sc = (t > 0.0f) ? __uint_as_float((tb + 0x007FFFFFu) & 0xFF800000u) : 1.0f;
         const uint32_t c = (uint32_t)f32_to_e4m3(v.x / sc) | ((uint32_t)f32_to_e4m3(v.y / sc) << 8) |
                            ((uint32_t)f32_to_e4m3(v.z / sc) << 16) | ((uint32_t)f32_to_e4m3(v.w / sc) << 24);
         *reinterpret_cast<uint32_t*>(o + b * 128 + 4 * lane) = c;

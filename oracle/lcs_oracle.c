@@ -131,7 +131,9 @@ ORC_API uint8_t orc_e2m1_code(double v)
 /* Mixed-precision KV row: dims [0, d_c) in E4M3 with one fp32 scale per
  * 128-dim block, dims [d_c, d_c + d_r) in bf16.  Row bytes:
  *   d_c codes | 2*d_r bytes bf16 | 4*(d_c/128) bytes fp32 scales.
- * scale = amax/448 in fp32 (1 if amax == 0); code = E4M3(x/scale), x/scale in fp32. */
+ * scale = the smallest power of two >= amax/448 (amax/448 in fp32; 1 if amax == 0),
+ * code = E4M3(x/scale).  With a power-of-two scale every stored value code*scale
+ * is exactly representable in bf16, so widening to bf16 loses nothing. */
 ORC_API void orc_quant_kv_fp8(const float* x, int64_t n, int d_c, int d_r, uint8_t* out)
 {
     int nb = d_c / 128;
@@ -145,8 +147,14 @@ ORC_API void orc_quant_kv_fp8(const float* x, int64_t n, int d_c, int d_r, uint8
                 float a = fabsf(xr[b * 128 + j]);
                 if (a > amax) amax = a;
             }
-            float sc = amax / 448.0f;
-            if (sc == 0.0f) sc = 1.0f;
+            float t = amax / 448.0f;
+            float sc = 1.0f;
+            if (t > 0.0f) {
+                int e;
+                float f = frexpf(t, &e);            /* t = f * 2^e, 0.5 <= f < 1 */
+                sc = (f == 0.5f) ? t : ldexpf(1.0f, e);
+                if (sc < 0x1p-126f) sc = 0x1p-126f;   /* at least the smallest normal */
+            }
             for (int j = 0; j < 128; ++j) {
                 float t = xr[b * 128 + j] / sc;
                 o[b * 128 + j] = orc_e4m3_code(orc_round_e4m3((double)t));
