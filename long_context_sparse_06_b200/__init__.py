@@ -205,12 +205,12 @@ def _attend_common(q, comp, win, kv_dtype, d_v):
 
 
 def csa_attend(q, comp, win, idx, d_v, scale, kv_dtype=None, q_pos=None, win_pos0=None, W=128, want_lse=False,
-               ws=None, stream=None):
+               out_dtype=None, ws=None, stream=None):
     """q [B,Q,H,D]; comp [B,N_c,row]; win [B,Tw,row]; idx [B,Q,k] -> out [B,Q,H,d_v] (and lse)."""
     torch = _torch()
     B, Q, H, D, kv_dtype, N_c, Tw = _attend_common(q, comp, win, kv_dtype, d_v)
     k = idx.shape[-1]
-    out = torch.empty((B, Q, H, d_v), dtype=q.dtype, device=q.device)
+    out = torch.empty((B, Q, H, d_v), dtype=out_dtype or q.dtype, device=q.device)
     lse = torch.empty((B, Q, H), dtype=torch.float32, device=q.device) if want_lse else None
     if ws is None:
         ws = workspace(lcs_workspace_size(OP_ATTEND, B, Q, N_c, Tw, k, H, d_v), q.device)
@@ -220,10 +220,10 @@ def csa_attend(q, comp, win, idx, d_v, scale, kv_dtype=None, q_pos=None, win_pos
 
 
 def hca_attend(q, comp, win, d_v, scale, kv_dtype=None, q_pos=None, win_pos0=None, m=128, W=128, want_lse=False,
-               ws=None, stream=None):
+               out_dtype=None, ws=None, stream=None):
     torch = _torch()
     B, Q, H, D, kv_dtype, N_c, Tw = _attend_common(q, comp, win, kv_dtype, d_v)
-    out = torch.empty((B, Q, H, d_v), dtype=q.dtype, device=q.device)
+    out = torch.empty((B, Q, H, d_v), dtype=out_dtype or q.dtype, device=q.device)
     lse = torch.empty((B, Q, H), dtype=torch.float32, device=q.device) if want_lse else None
     if ws is None:
         ws = workspace(lcs_workspace_size(OP_ATTEND, B, Q, N_c, Tw, 0, H, d_v), q.device)
@@ -234,7 +234,7 @@ def hca_attend(q, comp, win, d_v, scale, kv_dtype=None, q_pos=None, win_pos0=Non
 
 
 def decode_fused(mode, q, comp, win, d_v, scale, kv_dtype=None, qI=None, w=None, kI=None, kI_dtype=None, k=0,
-                 score_dtype=None, out=None, want_lse=False, idx_out=None, ws=None, stream=None):
+                 score_dtype=None, out=None, out_dtype=None, want_lse=False, idx_out=None, ws=None, stream=None):
     """One decode step (Q = 1 per request).  q [B,H,D]; comp [B,N_c,row]; win [B,Tw,row];
     CSA: qI [B,H_I,d_I], w [B,H_I], kI [B,N_c,d_I] or FP4 planes.  Returns out [B,H,d_v]."""
     torch = _torch()
@@ -256,7 +256,7 @@ def decode_fused(mode, q, comp, win, d_v, scale, kv_dtype=None, qI=None, w=None,
         kI_dtype = kI_dtype if kI_dtype is not None else F32
         score_dtype = score_dtype if score_dtype is not None else F32
     if out is None:
-        out = torch.empty((B, H, d_v), dtype=q.dtype, device=q.device)
+        out = torch.empty((B, H, d_v), dtype=out_dtype or q.dtype, device=q.device)
     lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if want_lse else None
     if ws is None:
         ws = workspace(lcs_workspace_size(OP_DECODE, B, 1, N_c, Tw, k, H, d_v, score_dtype), q.device)

@@ -179,7 +179,7 @@ static int validate_index(const void* qI, int qI_dtype, const float* w, const vo
                           int64_t Q, int64_t N_c, int H_I, int d_I, const int64_t* q_pos, int m, int k,
                           int score_dtype) {
     if (qI == nullptr || w == nullptr || kI == nullptr) return LCS_ERR_INVALID;
-    if (B < 0 || Q < 0 || N_c < 0 || H_I <= 0 || d_I <= 0 || d_I % 32 || k < 0 || k > 8192) return LCS_ERR_INVALID;
+    if (B < 0 || Q < 0 || N_c < 0 || H_I <= 0 || d_I <= 0 || d_I % 32 || k < 0 || k > 4096) return LCS_ERR_INVALID;
     if (q_pos == nullptr && Q != 1) return LCS_ERR_INVALID;
     if (q_pos != nullptr && m < 1) return LCS_ERR_INVALID;
     if (N_c >= (int64_t(1) << 31) || B * N_c >= (int64_t(1) << 31)) return LCS_ERR_INVALID;
@@ -234,7 +234,7 @@ int csa_index_topk(const void* qI, int qI_dtype, const float* w, const void* kI,
 int lcs_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, int64_t N_c, const int64_t* q_pos, int m,
              int k, int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
     if (scores == nullptr || idx == nullptr) return LCS_ERR_INVALID;
-    if (B < 0 || Q < 0 || N_c < 0 || k < 0 || k > 8192) return LCS_ERR_INVALID;
+    if (B < 0 || Q < 0 || N_c < 0 || k < 0 || k > 4096) return LCS_ERR_INVALID;
     if (q_pos != nullptr && m < 1) return LCS_ERR_INVALID;
     if (score_dtype != LCS_F32 && score_dtype != LCS_BF16) return LCS_ERR_UNSUPPORTED;
     if (ws == nullptr || ws_bytes < (size_t)kStatusBytes) return LCS_ERR_WORKSPACE;
@@ -258,7 +258,7 @@ static int validate_attend(const AttendArgs& a, int q_dtype, int out_dtype) {
         return LCS_OK;
     }
     if (a.kv_dtype == LCS_BF16 || a.kv_dtype == LCS_KV_FP8) {
-        if (q_dtype != LCS_BF16 || out_dtype != LCS_BF16) return LCS_ERR_UNSUPPORTED;
+        if (q_dtype != LCS_BF16 || (out_dtype != LCS_BF16 && out_dtype != LCS_F32)) return LCS_ERR_UNSUPPORTED;
         if (a.H != 64 || a.D != 576 || a.d_v != 512 || a.k > 2048) return LCS_ERR_UNSUPPORTED;
         if (!aligned16(a.q) || !aligned16(a.comp) || (a.win && !aligned16(a.win)) || !aligned16(a.out))
             return LCS_ERR_INVALID;
@@ -282,7 +282,8 @@ int csa_attend(const void* q, int q_dtype, const void* comp, const void* win, in
                int W, int H, int D, int d_v, float scale, void* out, int out_dtype, float* lse, void* ws,
                size_t ws_bytes, cudaStream_t stream) {
     if (idx == nullptr || k < 0) return LCS_ERR_INVALID;
-    AttendArgs a{q, comp, win, kv_dtype, B, Q, N_c, Tw, idx, k, q_pos, win_pos0, 1, W, H, D, d_v, scale, out, lse};
+    AttendArgs a{q, comp, win, kv_dtype, B, Q, N_c, Tw, idx, k, q_pos, win_pos0, 1, W, H, D, d_v, scale, out, lse,
+                 out_dtype};
     return run_attend(a, q_dtype, out_dtype, ws, ws_bytes, kStatusBytes, stream, false);
 }
 
@@ -290,7 +291,8 @@ int hca_attend(const void* q, int q_dtype, const void* comp, const void* win, in
                int64_t N_c, int64_t Tw, const int64_t* q_pos, const int64_t* win_pos0, int m, int W, int H, int D,
                int d_v, float scale, void* out, int out_dtype, float* lse, void* ws, size_t ws_bytes,
                cudaStream_t stream) {
-    AttendArgs a{q, comp, win, kv_dtype, B, Q, N_c, Tw, nullptr, 0, q_pos, win_pos0, m, W, H, D, d_v, scale, out, lse};
+    AttendArgs a{q, comp, win, kv_dtype, B, Q, N_c, Tw, nullptr, 0, q_pos, win_pos0, m, W, H, D, d_v, scale, out, lse,
+                 out_dtype};
     return run_attend(a, q_dtype, out_dtype, ws, ws_bytes, kStatusBytes, stream, false);
 }
 
@@ -323,7 +325,7 @@ int decode_fused(int mode, int64_t B, const void* q, int q_dtype, const void* co
         if (v != LCS_OK) return v;
     }
     AttendArgs a{q, comp, win, kv_dtype, B, 1, N_c, Tw, nullptr, csa ? k : 0, nullptr, nullptr, 1, 128, H, D, d_v,
-                 scale, out, lse};
+                 scale, out, lse, out_dtype};
     if (csa) a.idx = reinterpret_cast<const int32_t*>(1);   // placeholder for validation and the split plan
     int v = validate_attend(a, q_dtype, out_dtype);
     if (v != LCS_OK) return v;
@@ -396,7 +398,7 @@ int64_t lcs_workspace_size(int op, int64_t B, int64_t Q, int64_t N_c, int64_t Tw
         case LCS_OP_ATTEND: {
             // Upper bound over CSA (k rows) and HCA (N_c rows); the window counted as Tw rows.
             AttendArgs a{nullptr, nullptr, nullptr, LCS_BF16, B, Q, N_c, Tw, nullptr, k, nullptr, nullptr, 1, 128,
-                         H, 576, d_v, 1.f, nullptr, nullptr};
+                         H, 576, d_v, 1.f, nullptr, nullptr, LCS_BF16};
             AttendArgs c = a;
             c.idx = reinterpret_cast<const int32_t*>(1);
             int64_t s1 = attend_scratch_bytes(a), s2 = attend_scratch_bytes(c);
@@ -404,7 +406,7 @@ int64_t lcs_workspace_size(int op, int64_t B, int64_t Q, int64_t N_c, int64_t Tw
         }
         case LCS_OP_DECODE: {
             AttendArgs a{nullptr, nullptr, nullptr, LCS_BF16, B, 1, N_c, Tw, nullptr, k, nullptr, nullptr, 1, 128,
-                         H, 576, d_v, 1.f, nullptr, nullptr};
+                         H, 576, d_v, 1.f, nullptr, nullptr, LCS_BF16};
             AttendArgs c = a;
             c.idx = reinterpret_cast<const int32_t*>(1);
             int64_t so, io, ao;

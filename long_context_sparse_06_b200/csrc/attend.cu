@@ -40,7 +40,6 @@ constexpr int kH = 64, kD = 576, kDv = 512, kChunk = 64;
 constexpr int kBlk = kChunk * 128;            // one SW128 column block of a chunk: 64 rows x 128 B
 constexpr int kStageBytes = 9 * kBlk;         // 72 KB
 constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
-constexpr int kMaxK = 2048;
 constexpr int kAtThreads = 288;
 constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kBlk;   // + the P_lo buffer
 constexpr float kLog2e = 1.4426950408889634f;
@@ -86,7 +85,7 @@ __device__ __forceinline__ RowPlan plan_rows(const AttendArgs& a, int64_t g, int
 __device__ __forceinline__ const uint8_t* row_ptr(const AttendArgs& a, int64_t b, const RowPlan& p,
                                                   const int32_t* sel, int64_t r, int row_bytes) {
     if (r < p.nsel) {
-        const int64_t e = sel ? __ldg(sel + r) : r;
+        const int64_t e = sel ? sel[r] : r;   // sel may be global (tensor-core path) or shared (fp32 path)
         return static_cast<const uint8_t*>(a.comp) + (b * a.N_c + e) * row_bytes;
     }
     return static_cast<const uint8_t*>(a.win) + (b * a.Tw + p.win_lo + (r - p.nsel)) * row_bytes;
@@ -216,59 +215,67 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
         }
     } else if (warp >= 4) {
-        // ---------------- gather producer: warps 4..7 (128 threads)
-        const int pt = threadIdx.x - 128;
+        // ---------------- gather producer: warps 4..7.  Warp pw owns rows pw, pw+4, ..., pw+60 of
+        // a chunk; lane i first resolves the source of row pw+4i (one index load per row), then
+        // the warp streams each row with lanes on consecutive 16-byte pieces (coalesced).
+        const int pw = warp - 4;
         for (int c = 0; c < nch; ++c) {
             const int st = c & 1;
             if (c >= 2 && !mbar_wait(&bars.kempty[st], (uint32_t)(((c - 2) >> 1) & 1), status, 310)) break;
             uint8_t* dst = stage_s + st * kStageBytes;
             const int64_t r0 = (c_begin + c) * kChunk;
-            if constexpr (!FP8) {
-                // 64 rows x 72 chunks of 16 B; thread pt takes chunks pt, pt+128, ...
-                for (int i = pt; i < kChunk * 72; i += 128) {
-                    const int rr = i / 72, ch = i - rr * 72;
-                    const int64_t r = r0 + rr;
-                    const bool valid = r < R;
-                    const uint8_t* src = valid ? row_ptr(a, b, plan, sel, r, row_bytes) + ch * 16
-                                               : static_cast<const uint8_t*>(a.win);
-                    cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), src, valid);
-                }
-                cp_async_commit();
-                cp_async_wait<0>();
-            } else {
-                // FP8 rows: 32 content segments of 16 codes + 8 RoPE chunks of 8 bf16 per row
-                for (int i = pt; i < kChunk * 40; i += 128) {
-                    const int rr = i / 40, seg = i - rr * 40;
-                    const int64_t r = r0 + rr;
-                    uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-                    if (r < R) {
-                        const uint8_t* src = row_ptr(a, b, plan, sel, r, row_bytes);
-                        if (seg < 32) {
-                            const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + seg * 16));
-                            const float sc = __ldg(reinterpret_cast<const float*>(src + 640) + (seg >> 3));
-                            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                            uint32_t o[8];
+            const uint8_t* my_src = nullptr;
+            if (lane < 16) {
+                const int64_t r = r0 + pw + 4 * lane;
+                if (r < R) my_src = row_ptr(a, b, plan, sel, r, row_bytes);
+            }
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const int rr = pw + 4 * i;
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(
+                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), i));
+                const bool valid = src != nullptr;
+                if constexpr (!FP8) {
+                    const uint8_t* base = valid ? src : static_cast<const uint8_t*>(a.comp);
+                    for (int ch = lane; ch < 72; ch += 32)
+                        cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), base + (valid ? ch * 16 : 0), valid);
+                } else {
+                    // FP8 row: 32 content pieces of 16 codes (-> 32 bf16) and 8 RoPE pieces of 8 bf16
+                    for (int seg = lane; seg < 40; seg += 32) {
+                        uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+                        if (valid) {
+                            if (seg < 32) {
+                                const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + seg * 16));
+                                const float sc = __ldg(reinterpret_cast<const float*>(src + 640) + (seg >> 3));
+                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                                uint32_t o[8];
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                o[2 * q] = pack_bf16x2(e4m3_to_f32(w[q] & 0xFF) * sc, e4m3_to_f32((w[q] >> 8) & 0xFF) * sc);
-                                o[2 * q + 1] =
-                                    pack_bf16x2(e4m3_to_f32((w[q] >> 16) & 0xFF) * sc, e4m3_to_f32(w[q] >> 24) * sc);
+                                for (int q = 0; q < 4; ++q) {
+                                    o[2 * q] = pack_bf16x2(e4m3_to_f32(w4[q] & 0xFF) * sc,
+                                                           e4m3_to_f32((w4[q] >> 8) & 0xFF) * sc);
+                                    o[2 * q + 1] = pack_bf16x2(e4m3_to_f32((w4[q] >> 16) & 0xFF) * sc,
+                                                               e4m3_to_f32(w4[q] >> 24) * sc);
+                                }
+                                lo = make_uint4(o[0], o[1], o[2], o[3]);
+                                hi = make_uint4(o[4], o[5], o[6], o[7]);
+                            } else {
+                                lo = __ldg(reinterpret_cast<const uint4*>(src + 512 + (seg - 32) * 16));
                             }
-                            lo = make_uint4(o[0], o[1], o[2], o[3]);
-                            hi = make_uint4(o[4], o[5], o[6], o[7]);
+                        }
+                        if (seg < 32) {
+                            const int ch = seg * 2;
+                            *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
+                            *reinterpret_cast<uint4*>(dst + ((ch + 1) >> 3) * kBlk + sw128_off(rr, (ch + 1) & 7)) = hi;
                         } else {
-                            lo = __ldg(reinterpret_cast<const uint4*>(src + 512 + (seg - 32) * 16));
+                            const int ch = 64 + (seg - 32);
+                            *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
                         }
                     }
-                    if (seg < 32) {
-                        const int ch = seg * 2;   // two 16-byte bf16 chunks
-                        *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
-                        *reinterpret_cast<uint4*>(dst + ((ch + 1) >> 3) * kBlk + sw128_off(rr, (ch + 1) & 7)) = hi;
-                    } else {
-                        const int ch = 64 + (seg - 32);
-                        *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
-                    }
                 }
+            }
+            if constexpr (!FP8) {
+                cp_async_commit();
+                cp_async_wait<0>();
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars.kfull[st]);
@@ -368,7 +375,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const int dim0 = lo_half ? 0 : 256;
         if (splits == 1) {
             const float inv = (l_h > 0.f) ? 1.f / l_h : 0.f;
-            uint16_t* o = static_cast<uint16_t*>(a.out) + (g * kH + head) * kDv + dim0;
             for (int j = 0; j < 256 / 16; ++j) {
                 uint32_t ov[16];
                 if (have) {
@@ -378,12 +384,22 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 16; ++q) ov[q] = 0;
                 }
-                uint32_t pk[8];
+                if (a.out_dtype == LCS_F32) {
+                    float* o = static_cast<float*>(a.out) + (g * kH + head) * kDv + dim0 + j * 16;
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    pk[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
-                reinterpret_cast<uint4*>(o + j * 16)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                reinterpret_cast<uint4*>(o + j * 16)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    for (int q = 0; q < 4; ++q)
+                        reinterpret_cast<float4*>(o)[q] =
+                            make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
+                                        __uint_as_float(ov[4 * q + 2]) * inv, __uint_as_float(ov[4 * q + 3]) * inv);
+                } else {
+                    uint16_t* o = static_cast<uint16_t*>(a.out) + (g * kH + head) * kDv + dim0 + j * 16;
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        pk[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
+                    reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
             }
             if (a.lse != nullptr && lo_half)
                 a.lse[g * kH + head] = (l_h > 0.f) ? (m_h + log2f(l_h)) / kLog2e : -INFINITY;
@@ -421,7 +437,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 // Merges the split partials of each (query, head) in split order (fixed tree:
 // sequential), writing bf16 output and the natural-log LSE.
 __global__ void attend_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                      int splits, void* __restrict__ out, float* __restrict__ lse) {
+                                      int splits, void* __restrict__ out, int out_dtype, float* __restrict__ lse) {
     const int64_t gh = blockIdx.x;   // (query, head)
     float M = -INFINITY;
     for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[(gh / kH * splits + s) * kH * 2 + (gh % kH) * 2]);
@@ -438,7 +454,8 @@ __global__ void attend_combine_kernel(const float* __restrict__ part_o, const fl
             if (ml[1] > 0.f)
                 acc += part_o[((gh / kH * splits + s) * kH + gh % kH) * kDv + d] * exp2f(ml[0] - M);
         }
-        static_cast<uint16_t*>(out)[gh * kDv + d] = f32_to_bf16_bits(acc * inv);
+        if (out_dtype == LCS_F32) static_cast<float*>(out)[gh * kDv + d] = acc * inv;
+        else static_cast<uint16_t*>(out)[gh * kDv + d] = f32_to_bf16_bits(acc * inv);
     }
     if (lse != nullptr && threadIdx.x == 0) lse[gh] = L > 0.f ? (M + log2f(L)) / kLog2e : -INFINITY;
 }
@@ -582,7 +599,8 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
     e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, a, splits, part_o,
                  part_ml, status);
     if (e != cudaSuccess || splits == 1) return e;
-    attend_combine_kernel<<<(unsigned)(queries * kH), 128, 0, s>>>(part_o, part_ml, splits, a.out, a.lse);
+    attend_combine_kernel<<<(unsigned)(queries * kH), 128, 0, s>>>(part_o, part_ml, splits, a.out, a.out_dtype,
+                                                                    a.lse);
     return cudaGetLastError();
 }
 

@@ -61,6 +61,7 @@ struct AttendArgs {
     float scale;
     void* out;
     float* lse;
+    int out_dtype;   // LCS_F32 or LCS_BF16
 };
 int64_t attend_scratch_bytes(const AttendArgs& a);
 cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaStream_t s, bool pdl);
