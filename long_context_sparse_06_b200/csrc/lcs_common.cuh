@@ -83,16 +83,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete.  Returns false (and
 // records LCS_ERR_TIMEOUT with `where` as detail) if it does not within the
 // budget.  Once any wait in the grid has failed (status non-zero) later waits
-// give up immediately so that every thread reaches its exit path quickly.
+// give up at their next check so that every thread reaches its exit path.  The
+// clock and the status word (global memory) are consulted only every 64 polls,
+// so that a wait that is about to succeed is never held up by a memory round trip.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int where) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    while (true) {
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (status != nullptr && *(volatile int*)status != 0) return false;
-        if (globaltimer() - t0 > kWaitBudgetNs) {
-            set_status(status, LCS_ERR_TIMEOUT, where);
-            return false;
+        if ((it & 63u) == 0) {
+            if (status != nullptr && *(volatile int*)status != 0) return false;
+            if (globaltimer() - t0 > kWaitBudgetNs) {
+                set_status(status, LCS_ERR_TIMEOUT, where);
+                return false;
+            }
         }
     }
 }

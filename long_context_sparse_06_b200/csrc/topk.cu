@@ -10,19 +10,21 @@
 // element is ranked by the 64-bit composite (key << 32 | ~index), so "larger
 // composite" is exactly "larger score, then lower index".
 //
-// One CTA of 1024 threads per query row:
-//  1. Sample: a fixed strided sample of the row is bitonic-sorted in shared
-//     memory; its element of rank r (r chosen well below the sample's expected
-//     count above the true threshold) is a lower bound T for the k-th score.
-//  2. Filter: the row is read once; each warp walks its own contiguous segment
-//     and appends the composites with key >= T to its private candidate buffer,
-//     slots from __ballot_sync / __popc (no atomics, no contention).
-//  3. The candidates (typically ~2.5 k) are compacted and bitonic-sorted; the
-//     first k are the selection; their indices are bitonic-sorted ascending.
-// Rows no longer than the candidate capacity skip step 1.  If the bound misses
-// (fewer than k candidates, or a buffer overflows) the row falls back to an
-// exact MSB-first radix select (8-bit digits, shared-memory histograms) followed
-// by an ordered ballot compaction.  Every step is deterministic.
+// One CTA of 1024 threads per query row, three coalesced passes over the row:
+//  1. Histogram of the top 14 bits of every key (sign, exponent and the top
+//     mantissa bits of the score) in shared memory; the bins are fine enough
+//     that the 32 lanes of a warp rarely collide on one counter.  A block-wide
+//     suffix scan finds the bin holding the k-th largest score: every key in a
+//     higher bin is selected, and `need` more come from the threshold bin.
+//  2. The threshold bin's elements are gathered in index order (each warp walks
+//     its own contiguous segment; slots from __ballot_sync / __popc) and ranked
+//     exactly by counting, on the composite key.
+//  3. Ordered compaction: each warp re-walks its segment and writes the selected
+//     indices at offsets from ballots, so the output is ascending without a sort.
+// If the threshold bin is too crowded for the counting rank (massive ties) the
+// row falls back to an exact MSB-first radix select (8-bit digits, shared-memory
+// histograms) followed by the same kind of ordered compaction.  The result does
+// not depend on the order of the shared atomics, so every step is deterministic.
 #include <utility>
 
 #include "lcs_common.cuh"
@@ -34,47 +36,26 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kCandCap = 8192;                 // total candidate capacity
-constexpr int kWarpCap = kCandCap / kWarps;    // per-warp candidate buffer
-constexpr int kSampleMax = 4096;
+constexpr int kBinBits = 14;
+constexpr int kBins = 1 << kBinBits;
+constexpr int kCandCap = 2048;                 // threshold-bin elements ranked by counting
+constexpr int kWarpCap = 256;                  // per-warp gather buffer
 
 struct TopkSmem {
-    unsigned long long cand[kCandCap];      // per-warp candidate buffers, then the compacted sort array
-    unsigned long long sorted[kCandCap];    // compacted candidates (bitonic-sorted)
-    uint32_t sample[kSampleMax];            // sample keys; later the k selected indices
-    uint32_t hist[256], scan[256];
-    uint32_t warp_cnt[kWarps], warp_off[kWarps];
-    uint32_t digit, krem, total, fail;
+    uint32_t bins[kBins];                       // 64 KB histogram
+    unsigned long long wbuf[kWarps * kWarpCap]; // per-warp gather buffers (64 KB)
+    unsigned long long cand[kCandCap];          // threshold-bin candidates in index order
+    uint8_t take[kCandCap];                     // candidate selected?
+    uint32_t hist[256], scan[256];              // radix fallback
+    uint32_t warp_cnt[kWarps], warp_off[kWarps], warp_gt[kWarps], warp_sel[kWarps];
+    uint32_t wsum[kWarps];
+    uint32_t digit, krem, tbin, above, fail;
 };
 
 template <bool BF16>
 __device__ __forceinline__ uint32_t load_key(const void* row, int64_t i) {
     if constexpr (BF16) return bf16_key(static_cast<const uint16_t*>(row)[i]);
     else return f32_key(static_cast<const float*>(row)[i]);
-}
-
-// Bitonic sort of n (power of two) elements in shared memory, descending when
-// desc, by the whole block.
-template <typename T>
-__device__ void bitonic_sort(T* a, int n, bool desc) {
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = threadIdx.x; t < (n >> 1); t += blockDim.x) {
-                const int i = 2 * t - (t & (stride - 1));
-                const int j = i + stride;
-                const bool up = ((i & size) == 0) == desc;   // this pair's block is ordered "desc" when up
-                const T x = a[i], y = a[j];
-                if ((x < y) == up) { a[i] = y; a[j] = x; }
-            }
-            __syncthreads();
-        }
-    }
-}
-
-__device__ __forceinline__ int next_pow2(int x) {
-    int p = 1;
-    while (p < x) p <<= 1;
-    return p;
 }
 
 // ---------------------------------------------------------- exact fallback
@@ -155,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
                                                            int32_t* __restrict__ idx_out) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+    constexpr int kShift = (BF16 ? 16 : 32) - kBinBits;
     const int64_t row = blockIdx.x;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     int64_t n = N_c;
@@ -174,68 +156,114 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
         return;
     }
 
-    // ---- 1. lower bound from a sorted strided sample
-    uint32_t T = 0;
-    if (n > kCandCap) {
-        const int S = n <= 65536 ? 2048 : kSampleMax;
-        for (int i = t; i < S; i += kThreads) sm.sample[i] = load_key<BF16>(srow, (int64_t)i * n / S);
-        __syncthreads();
-        bitonic_sort(sm.sample, S, true);
-        int r = (int)((3 * (int64_t)k * S) / (2 * n)) + 8;   // 1.5x the expected rank of the k-th score, + 8
-        if (r > S - 1) r = S - 1;
-        T = sm.sample[r];
+    // ---- 1. histogram of the top bits, then the threshold bin by a suffix scan
+    for (int i = t; i < kBins; i += kThreads) sm.bins[i] = 0;
+    __syncthreads();
+    for (int64_t i = t; i < n; i += kThreads) atomicAdd(&sm.bins[load_key<BF16>(srow, i) >> kShift], 1u);
+    __syncthreads();
+    constexpr int kPer = kBins / kThreads;      // bins per thread, thread 0 owns the top ones
+    const int hi_bin = kBins - 1 - t * kPer;
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) local += sm.bins[hi_bin - j];
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
     }
+    if (lane == 31) sm.wsum[warp] = incl;
+    __syncthreads();
+    uint32_t wbase = 0;
+    for (int w = 0; w < warp; ++w) wbase += sm.wsum[w];
+    const uint32_t excl = wbase + incl - local;
+    if (excl < (uint32_t)k && excl + local >= (uint32_t)k) {
+        uint32_t run = excl;
+        for (int j = 0; j < kPer; ++j) {
+            const uint32_t c = sm.bins[hi_bin - j];
+            if (run + c >= (uint32_t)k) { sm.tbin = hi_bin - j; sm.above = run; break; }
+            run += c;
+        }
+    }
+    __syncthreads();
+    const uint32_t tbin = sm.tbin, above = sm.above, need = (uint32_t)k - above;
+    const uint32_t m_t = sm.bins[tbin];          // elements in the threshold bin
 
-    // ---- 2. filter into per-warp buffers (warp w owns a contiguous segment)
+    // ---- 2. gather the threshold bin in index order; count the keys above it
     const int64_t seg = ((n + kWarps - 1) / kWarps + 31) / 32 * 32;
     const int64_t s0 = warp * seg, s1 = (s0 + seg < n) ? s0 + seg : n;
-    unsigned long long* wbuf = sm.cand + warp * kWarpCap;
-    uint32_t cnt = 0;
     const uint32_t lt = (1u << lane) - 1u;
-    for (int64_t base = s0; base < s1; base += 32) {
-        const int64_t i = base + lane;
-        const bool act = i < s1;
-        const uint32_t key = act ? load_key<BF16>(srow, i) : 0u;
-        const bool keep = act && key >= T;
-        const uint32_t mk = __ballot_sync(0xffffffffu, keep);
-        const uint32_t slot = cnt + __popc(mk & lt);
-        if (keep && slot < kWarpCap)
-            wbuf[slot] = ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)i);
-        cnt += __popc(mk);
+    unsigned long long* wb = sm.wbuf + warp * kWarpCap;
+    uint32_t cnt = 0, gt = 0;
+    if (m_t <= kCandCap) {
+        for (int64_t base = s0; base < s1; base += 32) {
+            const int64_t i = base + lane;
+            const bool act = i < s1;
+            const uint32_t key = act ? load_key<BF16>(srow, i) : 0u;
+            const uint32_t bn = key >> kShift;
+            const bool eq = act && bn == tbin;
+            const uint32_t em = __ballot_sync(0xffffffffu, eq);
+            const uint32_t slot = cnt + __popc(em & lt);
+            if (eq && slot < kWarpCap)
+                wb[slot] = ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)i);
+            cnt += __popc(em);
+            gt += __popc(__ballot_sync(0xffffffffu, act && bn > tbin));
+        }
     }
-    if (lane == 0) sm.warp_cnt[warp] = cnt;
+    if (lane == 0) { sm.warp_cnt[warp] = cnt; sm.warp_gt[warp] = gt; }
     __syncthreads();
     if (t == 0) {
-        uint32_t off = 0, fail = 0;
+        uint32_t off = 0, fail = m_t > kCandCap;
         for (int w = 0; w < kWarps; ++w) {
             sm.warp_off[w] = off;
             off += sm.warp_cnt[w];
             fail |= sm.warp_cnt[w] > (uint32_t)kWarpCap;
         }
-        sm.total = off;
-        sm.fail = fail || off < (uint32_t)k;
+        sm.fail = fail;
     }
     __syncthreads();
     if (sm.fail) {
         radix_select<BF16>(sm, srow, n, k, out);
         return;
     }
+    for (uint32_t j = lane; j < cnt; j += 32) sm.cand[sm.warp_off[warp] + j] = wb[j];
+    __syncthreads();
 
-    // ---- 3. compact, sort descending, take k, sort their indices ascending
-    const int C = (int)sm.total;
-    const int P = next_pow2(C);
-    for (int w = warp; w < kWarps; w += kWarps) {
-        const uint32_t c = sm.warp_cnt[w], o = sm.warp_off[w];
-        for (uint32_t j = lane; j < c; j += 32) sm.sorted[o + j] = sm.cand[w * kWarpCap + j];
+    // ---- rank the threshold bin by counting (composite keys are distinct)
+    for (uint32_t j = t; j < m_t; j += kThreads) {
+        const unsigned long long c = sm.cand[j];
+        uint32_t r = 0;
+        for (uint32_t i = 0; i < m_t; ++i) r += sm.cand[i] > c;
+        sm.take[j] = r < need;
     }
-    for (int i = C + t; i < P; i += kThreads) sm.sorted[i] = 0ull;
     __syncthreads();
-    bitonic_sort(sm.sorted, P, true);
-    const int Pk = next_pow2(k);
-    for (int i = t; i < Pk; i += kThreads) sm.sample[i] = (i < k) ? ~(uint32_t)(sm.sorted[i] & 0xFFFFFFFFull) : 0xFFFFFFFFu;
+    {   // selected candidates per warp segment
+        const uint32_t o = sm.warp_off[warp];
+        uint32_t c = 0;
+        for (uint32_t j = lane; j < cnt; j += 32) c += sm.take[o + j];
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) c += __shfl_xor_sync(0xffffffffu, c, x);
+        if (lane == 0) sm.warp_sel[warp] = c;
+    }
     __syncthreads();
-    bitonic_sort(sm.sample, Pk, false);
-    for (int i = t; i < k; i += kThreads) out[i] = (int32_t)sm.sample[i];
+
+    // ---- 3. ordered compaction
+    uint32_t pos = 0;
+    for (int w = 0; w < warp; ++w) pos += sm.warp_gt[w] + sm.warp_sel[w];
+    uint32_t ci = sm.warp_off[warp];
+    for (int64_t base = s0; base < s1; base += 32) {
+        const int64_t i = base + lane;
+        const bool act = i < s1;
+        const uint32_t key = act ? load_key<BF16>(srow, i) : 0u;
+        const uint32_t bn = key >> kShift;
+        const bool eq = act && bn == tbin;
+        const uint32_t em = __ballot_sync(0xffffffffu, eq);
+        const bool tk = (act && bn > tbin) || (eq && sm.take[ci + __popc(em & lt)]);
+        const uint32_t tm = __ballot_sync(0xffffffffu, tk);
+        if (tk) out[pos + __popc(tm & lt)] = (int32_t)i;
+        pos += __popc(tm);
+        ci += __popc(em);
+    }
 }
 
 }  // namespace

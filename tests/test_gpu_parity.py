@@ -108,14 +108,14 @@ def test_compress(L, orc, case):
 # --------------------------------------------------------------------- top-k
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_topk_bit_exact_on_same_scores(L, orc, dtype):
-    rows, N = 7, 5000
+    rows, N = 7, 3000
     s = randn("g.tk", (1, rows, N), std=4.0)
     s[0, 1] = torch.round(s[0, 1])                 # heavy ties
     s[0, 2] = 0.0
     s[0, 2, ::7] = -0.0                            # signed zeros tie with +0
     s[0, 3, 100:] = -1e30                          # almost all equal below the top
     s = s.to(dtype)
-    for k in (1, 64, 512, 1024, 4999, 5000, 6000):
+    for k in (1, 64, 512, 1024, 2999, 3000, 4000):
         idx = L.lcs_topk(s.to(DEV), k).cpu().numpy()
         for r in range(rows):
             ref = orc.topk(s[0, r].float().numpy(), k)
