@@ -88,16 +88,74 @@ int num_sms() {
     return g_sms > 0 ? g_sms : 148;
 }
 
+namespace {
+// Small cache of encoded tensor maps: decode loops call with the same buffers every
+// step, and encoding costs microseconds of host time per map.
+struct TmapKey {
+    int dt;
+    const void* base;
+    uint64_t inner, outer, stride;
+    uint32_t bi, bo;
+    int swz;
+    bool operator==(const TmapKey& o) const {
+        return dt == o.dt && base == o.base && inner == o.inner && outer == o.outer && stride == o.stride &&
+               bi == o.bi && bo == o.bo && swz == o.swz;
+    }
+};
+constexpr int kTmapCache = 32;
+TmapKey g_tkeys[kTmapCache];
+CUtensorMap g_tmaps[kTmapCache];
+int g_tnext = 0, g_tcount = 0;
+std::mutex g_tmutex;
+}  // namespace
+
+namespace {
+constexpr int kAttrSlots = 64;
+const void* g_attr_fn[kAttrSlots];
+size_t g_attr_bytes[kAttrSlots];
+int g_attr_n = 0;
+std::mutex g_attr_mutex;
+}  // namespace
+
+cudaError_t set_smem_once(const void* kern, size_t bytes) {
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    int i = 0;
+    for (; i < g_attr_n; ++i)
+        if (g_attr_fn[i] == kern) break;
+    if (i < g_attr_n && g_attr_bytes[i] >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    if (i == g_attr_n && g_attr_n < kAttrSlots) g_attr_fn[g_attr_n++] = kern;
+    if (i < kAttrSlots) g_attr_bytes[i] = bytes;
+    return cudaSuccess;
+}
+
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    const TmapKey key{(int)dt, base, inner, outer, row_stride_bytes, box_inner, box_outer, (int)swz};
+    {
+        std::lock_guard<std::mutex> lock(g_tmutex);
+        for (int i = 0; i < g_tcount; ++i)
+            if (g_tkeys[i] == key) {
+                *map = g_tmaps[i];
+                return true;
+            }
+    }
     EncodeTiledFn fn = get_encoder();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {row_stride_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lock(g_tmutex);
+    g_tkeys[g_tnext] = key;
+    g_tmaps[g_tnext] = *map;
+    g_tnext = (g_tnext + 1) % kTmapCache;
+    if (g_tcount < kTmapCache) ++g_tcount;
+    return true;
 }
 
 }  // namespace lcs

@@ -20,12 +20,12 @@
 //    cp.async (bf16) or load-convert-store (FP8 rows: E4M3 x block scale ->
 //    bf16), writing the SW128 layout that both MMAs read (the same bytes are
 //    the K-major B of Q.K^T and the MN-major B of P.V);
-//  * warps 0-3 run the online softmax on S (fp32, exp2) and write P as two bf16
-//    parts, P = P_hi + P_lo (P_hi into the chunk's RoPE column block, dead once
-//    Q.K^T has read it; P_lo into its own buffer), so P.V carries ~16 bits of P;
-//    they rescale O in TMEM only when a head's running max grows by more than
-//    2^8 in weight, and finally normalise O and write it out (or a split
-//    partial for the combine).
+//  * warps 0-3 run the online softmax on S (fp32, exp2; S double-buffered in
+//    TMEM so Q.K^T of the next chunk overlaps it), write P as bf16 into the
+//    chunk's RoPE column block (dead once Q.K^T has read it), rescale O in TMEM
+//    only when a head's running max grows by more than 2^8 in weight, and
+//    finally normalise O and write it out (or a split partial for the combine)
+//    through shared memory, so the global stores are coalesced.
 // F32 path (C1-sized problems): CUDA cores, fp32 online softmax.
 #include <utility>
 
@@ -40,17 +40,18 @@ constexpr int kH = 64, kD = 576, kDv = 512, kChunk = 64;
 constexpr int kBlk = kChunk * 128;            // one SW128 column block of a chunk: 64 rows x 128 B
 constexpr int kStageBytes = 9 * kBlk;         // 72 KB
 constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
-constexpr int kAtThreads = 288;
-constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kBlk;   // + the P_lo buffer
+constexpr int kAtThreads = 320;   // 4 softmax, 4 gather, 1 Q.K^T issuer, 1 P.V issuer
+constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
 
 struct AtBars {
     uint64_t qfull;
     uint64_t kfull[2], kempty[2];
-    uint64_t sfull, sempty;
+    uint64_t sfull[2], sempty[2];
     uint64_t pfull[2];
-    uint64_t ofull;
+    uint64_t ofull[2];   // P.V of chunk c done (per chunk parity)
+    uint64_t odone;      // every P.V of this CTA done
     uint32_t tmem_base;
     int nsel;
 };
@@ -100,7 +101,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* q_s = smem;
     uint8_t* stage_s = smem + kQBytes;
-    uint8_t* plo_s = smem + kQBytes + 2 * kStageBytes;   // P_lo [64 heads x 64 rows] bf16, SW128
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g = blockIdx.x / splits;
@@ -114,11 +114,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             mbar_init(&bars.kfull[i], 128);
             mbar_init(&bars.kempty[i], 1);
             mbar_init(&bars.pfull[i], 128);
+            mbar_init(&bars.sfull[i], 1);
+            mbar_init(&bars.sempty[i], 128);
+            mbar_init(&bars.ofull[i], 1);
         }
-        mbar_init(&bars.sfull, 1);
-        mbar_init(&bars.sempty, 128);
-        mbar_init(&bars.ofull, 1);
+        mbar_init(&bars.odone, 1);
         fence_barrier_init();
+        prefetch_tmap(&map_q);
     }
     if (warp == 8) {
         tmem_alloc(&bars.tmem_base, 512);
@@ -132,15 +134,25 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (a.idx != nullptr) {
         if (warp == 0) {
             const int32_t* ir = a.idx + g * a.k;
-            int n = a.k;
-            for (int base = 0; base < a.k && n == a.k; base += 32) {
-                const int i = base + lane;
-                const int32_t v = (i < a.k) ? ir[i] : 0;
-                if (i < a.k && v >= a.N_c) set_status(status, LCS_ERR_DEVICE, 201);
-                const uint32_t bad = __ballot_sync(0xffffffffu, i < a.k && (v < 0 || v >= a.N_c));
-                if (bad) n = base + __ffs(bad) - 1;
+            int first_bad = a.k;
+            for (int base = 0; base < a.k; base += 256) {
+                int32_t v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = base + 32 * j + lane;
+                    v[j] = (i < a.k) ? __ldg(ir + i) : 0;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = base + 32 * j + lane;
+                    if (i < a.k && (v[j] < 0 || v[j] >= a.N_c)) {
+                        if (v[j] >= a.N_c) set_status(status, LCS_ERR_DEVICE, 201);
+                        first_bad = min(first_bad, i);
+                    }
+                }
             }
-            if (lane == 0) bars.nsel = n;
+            first_bad = __reduce_min_sync(0xffffffffu, first_bad);
+            if (lane == 0) bars.nsel = first_bad;
         }
     } else if (threadIdx.x == 0) {
         int64_t n = a.N_c;
@@ -165,7 +177,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
     constexpr uint32_t idesc_qk = idesc_bf16(64, kChunk, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16(64, 256, false, true);
-    const uint32_t t_s = tmem + 256;   // S: columns 256..319, lanes of the M=64 layout
+    // TMEM: O in columns 0..255 (dims 0-255 at lane offset 0, dims 256-511 at lane
+    // offset 16: two interleaved M=64 accumulators), S double-buffered in 256..383.
+    auto t_s = [&](int buf) { return tmem + 256u + 64u * (uint32_t)buf; };
 
     if (warp == 8) {
         if (lane == 0 && nch > 0) {
@@ -174,45 +188,49 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             for (int blk = 0; blk < 9; ++blk)
                 tma_load_2d(q_s + blk * (kH * 128), &map_q, &bars.qfull, blk * 64, (int)(g * kH));
             bool ok = mbar_wait(&bars.qfull, 0, status, 300);
-            const uint32_t q_base = smem_u32(q_s);
+            // descriptors: base once, then byte offsets >> 4 added to the start-address field
+            const uint64_t q_desc = sw128_desc(smem_u32(q_s), 16, 1024);
+            const uint64_t k_desc0 = sw128_desc(smem_u32(stage_s), 16, 1024);
             auto issue_qk = [&](int c) -> bool {
                 const int st = c & 1;
                 if (!mbar_wait(&bars.kfull[st], (uint32_t)((c >> 1) & 1), status, 301)) return false;
-                if (c > 0 && !mbar_wait(&bars.sempty, (uint32_t)((c - 1) & 1), status, 302)) return false;
+                if (c >= 2 && !mbar_wait(&bars.sempty[st], (uint32_t)(((c - 2) >> 1) & 1), status, 302)) return false;
                 tc_fence_after();
-                const uint32_t k_base = smem_u32(stage_s + st * kStageBytes);
+                const uint64_t kd = k_desc0 + (uint64_t)((st * kStageBytes) >> 4);
+#pragma unroll
                 for (int blk = 0; blk < 9; ++blk)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = sw128_desc(q_base + blk * (kH * 128) + kk * 32, 16, 1024);
-                        const uint64_t bd = sw128_desc(k_base + blk * kBlk + kk * 32, 16, 1024);
-                        mma_bf16_ss(t_s, ad, bd, idesc_qk, (blk | kk) ? 1u : 0u);
-                    }
-                mma_commit(&bars.sfull);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(t_s(st), q_desc + (uint64_t)((blk * (kH * 128) + kk * 32) >> 4),
+                                    kd + (uint64_t)((blk * kBlk + kk * 32) >> 4), idesc_qk, (blk | kk) ? 1u : 0u);
+                mma_commit(&bars.sfull[st]);
                 return true;
             };
-            if (ok) ok = issue_qk(0);
-            for (int c = 0; c < nch && ok; ++c) {
-                if (c + 1 < nch) ok = issue_qk(c + 1);
-                if (!ok) break;
+            for (int c = 0; c < nch && ok; ++c) ok = issue_qk(c);
+        }
+    } else if (warp == 9) {
+        if (lane == 0 && nch > 0) {
+            // ---------------- P.V issue (its own thread, so that it never waits behind the
+            // next chunk's Q.K^T, which waits for that chunk's gather)
+            const uint64_t k_desc0 = sw128_desc(smem_u32(stage_s), 16, 1024);
+            const uint64_t v_desc0 = sw128_desc(smem_u32(stage_s), kBlk, 1024);
+            for (int c = 0; c < nch; ++c) {
                 const int st = c & 1;
-                if (!mbar_wait(&bars.pfull[st], (uint32_t)((c >> 1) & 1), status, 303)) { ok = false; break; }
+                if (!mbar_wait(&bars.pfull[st], (uint32_t)((c >> 1) & 1), status, 303)) break;
                 tc_fence_after();
-                const uint32_t phi_base = smem_u32(stage_s + st * kStageBytes + 8 * kBlk);
-                const uint32_t plo_base = smem_u32(plo_s);
-                const uint32_t v_base = smem_u32(stage_s + st * kStageBytes);
+                const uint64_t pd = k_desc0 + (uint64_t)((st * kStageBytes + 8 * kBlk) >> 4);
+                const uint64_t vd = v_desc0 + (uint64_t)((st * kStageBytes) >> 4);
 #pragma unroll
                 for (int half = 0; half < 2; ++half)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd = sw128_desc(v_base + half * 4 * kBlk + kk * 2048, kBlk, 1024);
-                        const uint32_t d_t = tmem + (half ? (16u << 16) : 0u);
-                        mma_bf16_ss(d_t, sw128_desc(phi_base + kk * 32, 16, 1024), bd, idesc_pv, (c | kk) ? 1u : 0u);
-                        mma_bf16_ss(d_t, sw128_desc(plo_base + kk * 32, 16, 1024), bd, idesc_pv, 1u);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + (half ? (16u << 16) : 0u), pd + (uint64_t)((kk * 32) >> 4),
+                                    vd + (uint64_t)((half * 4 * kBlk + kk * 2048) >> 4), idesc_pv,
+                                    (c | kk) ? 1u : 0u);
                 mma_commit(&bars.kempty[st]);
-                mma_commit(&bars.ofull);
+                mma_commit(&bars.ofull[st]);
             }
+            mma_commit(&bars.odone);
         }
     } else if (warp >= 4) {
         // ---------------- gather producer: warps 4..7.  Warp pw owns rows pw, pw+4, ..., pw+60 of
@@ -240,7 +258,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                     for (int ch = lane; ch < 72; ch += 32)
                         cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), base + (valid ? ch * 16 : 0), valid);
                 } else {
-                    // FP8 row: 32 content pieces of 16 codes (-> 32 bf16) and 8 RoPE pieces of 8 bf16
+                    // FP8 row: 32 content pieces of 16 codes (-> 32 bf16, exact with the
+                    // power-of-two block scale) and 8 RoPE pieces of 8 bf16
                     for (int seg = lane; seg < 40; seg += 32) {
                         uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
                         if (valid) {
@@ -281,33 +300,32 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             mbar_arrive(&bars.kfull[st]);
         }
     } else {
-        // ---------------- softmax / correction / epilogue: warps 0..3
-        const int quarter = warp;            // TMEM lanes 32*quarter .. +31
+        // ---------------- softmax / correction / epilogue: warps 0..3.  Warp q owns heads
+        // 16q..16q+15; lane l works on head 16q + (l & 15) and, with the 16x32bx2 TMEM
+        // load, on S columns 0-31 (lanes 0-15) or 32-63 (lanes 16-31).
+        const int quarter = warp;
         const int hl = lane & 15;
-        const int head = quarter * 16 + hl;  // head of this thread (both half-rows)
-        const bool lo_half = lane < 16;
-        float m_used = -INFINITY;            // log2-domain running max used for exponentials
-        float l_sum = 0.f;
+        const int head = quarter * 16 + hl;
+        const int cbase = (lane < 16) ? 0 : 32;   // this lane's S columns
+        float m_used = -INFINITY;                 // log2-domain running max used for exponentials
+        float l_sum = 0.f;                        // sum of the bf16-rounded weights (both lane halves)
         const float sl2 = a.scale * kLog2e;
         for (int c = 0; c < nch; ++c) {
             const int st = c & 1;
-            if (!mbar_wait(&bars.sfull, (uint32_t)(c & 1), status, 320)) break;
+            if (!mbar_wait(&bars.sfull[st], (uint32_t)((c >> 1) & 1), status, 320)) break;
             tc_fence_after();
-            uint32_t sv[kChunk];
-#pragma unroll
-            for (int j = 0; j < kChunk / 16; ++j)
-                tmem_ld16(tmem_addr(t_s, quarter * 32, j * 16), *reinterpret_cast<uint32_t(*)[16]>(&sv[j * 16]));
+            uint32_t sv[32];
+            tmem_ld16x2_32(tmem_addr(t_s(st), quarter * 32, 0), sv);
             tmem_ld_wait();
             tc_fence_before();
-            mbar_arrive(&bars.sempty);
+            mbar_arrive(&bars.sempty[st]);
             const int64_t rbase = (c_begin + c) * kChunk;
             const int nvalid = (int)((R - rbase) < kChunk ? (R - rbase) : kChunk);
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < kChunk; ++j)
-                if (j < nvalid) mx = fmaxf(mx, __uint_as_float(sv[j]) * sl2);
-            // lanes 16..31 read the unused upper half-lanes; take the max/decision of lane hl
-            mx = __shfl_sync(0xffffffffu, mx, hl);
+            for (int j = 0; j < 32; ++j)
+                if (cbase + j < nvalid) mx = fmaxf(mx, __uint_as_float(sv[j]) * sl2);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_used + kRescale || m_used == -INFINITY) {
@@ -316,21 +334,31 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 rescale = (c > 0);
                 m_used = m_new;
             }
-            // P = exp2(scale*s*log2e - m) of this thread's head (lanes 0..15 own the heads)
+            // P = bf16(exp2(scale*log2e*s - m)), written into the chunk's RoPE column block
+            // (dead once Q.K^T has read it): K-major SW128 rows of 128 B per head.
+            uint8_t* pblk = stage_s + st * kStageBytes + 8 * kBlk;
             float psum = 0.f;
-            if (lo_half) {
 #pragma unroll
-                for (int j = 0; j < kChunk; ++j) {
-                    const float p = (j < nvalid) ? exp2f(__uint_as_float(sv[j]) * sl2 - m_used) : 0.f;
-                    sv[j] = __float_as_uint(p);
-                    psum += p;
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int j = ch * 8 + 2 * q;
+                    const float p0 = (cbase + j < nvalid) ? exp2f(__uint_as_float(sv[j]) * sl2 - m_used) : 0.f;
+                    const float p1 = (cbase + j + 1 < nvalid) ? exp2f(__uint_as_float(sv[j + 1]) * sl2 - m_used) : 0.f;
+                    pk[q] = pack_bf16x2(p0, p1);
+                    psum += bf16_bits_to_f32((uint16_t)(pk[q] & 0xFFFF)) + bf16_bits_to_f32((uint16_t)(pk[q] >> 16));
                 }
+                *reinterpret_cast<uint4*>(pblk + sw128_off(head, (cbase >> 3) + ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
+            psum += __shfl_xor_sync(0xffffffffu, psum, 16);
             l_sum = l_sum * alpha + psum;
-            // P_lo and O are shared with the previous chunk's P.V: wait until it is done
-            if (c > 0 && !mbar_wait(&bars.ofull, (uint32_t)((c - 1) & 1), status, 321)) break;
-            tc_fence_after();
             if (__any_sync(0xffffffffu, rescale)) {
+                // O must be stable before it is rescaled: wait for the previous chunk's P.V.
+                // (P.V of chunk c-3 is complete here -- chunk c-1 was gathered after it -- so
+                // the per-chunk-parity barrier cannot be two phases behind.)
+                if (!mbar_wait(&bars.ofull[(c - 1) & 1], (uint32_t)(((c - 1) >> 1) & 1), status, 321)) break;
+                tc_fence_after();
                 const float f = rescale ? alpha : 1.f;
                 for (int j = 0; j < 256 / 16; ++j) {
                     uint32_t ov[16];
@@ -342,86 +370,72 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                     tmem_st16(ta, ov);
                 }
                 tmem_st_wait();
-            }
-            tc_fence_before();
-            // P_hi = bf16(P) into the chunk's RoPE block, P_lo = bf16(P - P_hi) into its buffer
-            // (K-major SW128 rows of 128 B per head)
-            if (lo_half) {
-                uint8_t* phi = stage_s + st * kStageBytes + 8 * kBlk;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t hi[4], lo[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float p0 = __uint_as_float(sv[ch * 8 + 2 * q]);
-                        const float p1 = __uint_as_float(sv[ch * 8 + 2 * q + 1]);
-                        hi[q] = pack_bf16x2(p0, p1);
-                        lo[q] = pack_bf16x2(p0 - bf16_bits_to_f32((uint16_t)(hi[q] & 0xFFFF)),
-                                            p1 - bf16_bits_to_f32((uint16_t)(hi[q] >> 16)));
-                    }
-                    *reinterpret_cast<uint4*>(phi + sw128_off(head, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    *reinterpret_cast<uint4*>(plo_s + sw128_off(head, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                }
+                tc_fence_before();
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars.pfull[st]);
         }
-        // ---- epilogue: O / l (or the split partial)
+        // ---- epilogue: O / l (or the split partial), staged through shared memory so that
+        // the global writes are coalesced.  Lane l of warp q holds O row of head 16q + (l & 15),
+        // dims 0-255 (lanes 0-15) or 256-511 (lanes 16-31).
         const bool have = nch > 0;
-        if (have && !mbar_wait(&bars.ofull, (uint32_t)((nch - 1) & 1), status, 322)) { /* fall through */ }
+        if (have) mbar_wait(&bars.odone, 0, status, 322);
         tc_fence_after();
-        const float l_h = __shfl_sync(0xffffffffu, l_sum, hl);
-        const float m_h = __shfl_sync(0xffffffffu, m_used, hl);
-        const int dim0 = lo_half ? 0 : 256;
-        if (splits == 1) {
-            const float inv = (l_h > 0.f) ? 1.f / l_h : 0.f;
-            for (int j = 0; j < 256 / 16; ++j) {
-                uint32_t ov[16];
-                if (have) {
-                    tmem_ld16(tmem_addr(tmem, quarter * 32, j * 16), ov);
-                    tmem_ld_wait();
-                } else {
+        const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
+        const int dim0 = (lane < 16) ? 0 : 256;
+        const bool final_out = splits == 1;
+        const bool f32 = !final_out || a.out_dtype == LCS_F32;
+        const int row_pitch = f32 ? (kDv * 4 + 16) : (kDv * 2 + 16);   // padded rows: fewer bank conflicts
+        uint8_t* ostage = stage_s;                                     // stages are free after the last P.V
+        const float fs = final_out ? inv : 1.f;
+        uint8_t* rowp = ostage + head * row_pitch;
+        for (int j0 = 0; j0 < 256 / 16; j0 += 4) {
+            uint32_t ov[4][16];
+            if (have) {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) ov[q] = 0;
-                }
-                if (a.out_dtype == LCS_F32) {
-                    float* o = static_cast<float*>(a.out) + (g * kH + head) * kDv + dim0 + j * 16;
+                for (int u = 0; u < 4; ++u) tmem_ld16(tmem_addr(tmem, quarter * 32, (j0 + u) * 16), ov[u]);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) ov[u][q] = 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u;
+                if (f32) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        reinterpret_cast<float4*>(o)[q] =
-                            make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
-                                        __uint_as_float(ov[4 * q + 2]) * inv, __uint_as_float(ov[4 * q + 3]) * inv);
+                        reinterpret_cast<float4*>(rowp + (dim0 + j * 16) * 4)[q] =
+                            make_float4(__uint_as_float(ov[u][4 * q]) * fs, __uint_as_float(ov[u][4 * q + 1]) * fs,
+                                        __uint_as_float(ov[u][4 * q + 2]) * fs, __uint_as_float(ov[u][4 * q + 3]) * fs);
                 } else {
-                    uint16_t* o = static_cast<uint16_t*>(a.out) + (g * kH + head) * kDv + dim0 + j * 16;
                     uint32_t pk[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        pk[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
-                    reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        pk[q] = pack_bf16x2(__uint_as_float(ov[u][2 * q]) * fs, __uint_as_float(ov[u][2 * q + 1]) * fs);
+                    reinterpret_cast<uint4*>(rowp + (dim0 + j * 16) * 2)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    reinterpret_cast<uint4*>(rowp + (dim0 + j * 16) * 2)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
-            if (a.lse != nullptr && lo_half)
-                a.lse[g * kH + head] = (l_h > 0.f) ? (m_h + log2f(l_h)) / kLog2e : -INFINITY;
-        } else {
-            float* po = part_o + ((g * splits + sp) * kH + head) * kDv + dim0;
-            for (int j = 0; j < 256 / 16; ++j) {
-                uint32_t ov[16];
-                if (have) {
-                    tmem_ld16(tmem_addr(tmem, quarter * 32, j * 16), ov);
-                    tmem_ld_wait();
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) ov[q] = 0;
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    reinterpret_cast<uint4*>(po + j * 16)[q] = make_uint4(ov[4 * q], ov[4 * q + 1], ov[4 * q + 2], ov[4 * q + 3]);
-            }
-            if (lo_half) {
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 epilogue warps
+        const int row_bytes_out = f32 ? kDv * 4 : kDv * 2;
+        uint8_t* gout = final_out ? static_cast<uint8_t*>(a.out) + g * kH * row_bytes_out
+                                  : reinterpret_cast<uint8_t*>(part_o + (g * splits + sp) * kH * kDv);
+        const int t128 = threadIdx.x;   // 0..127
+        for (int off = t128 * 16; off < kH * row_bytes_out; off += 128 * 16) {
+            const int h = off / row_bytes_out, cb = off - h * row_bytes_out;
+            *reinterpret_cast<uint4*>(gout + off) = *reinterpret_cast<const uint4*>(ostage + h * row_pitch + cb);
+        }
+        if (lane < 16) {
+            if (final_out) {
+                if (a.lse != nullptr) a.lse[g * kH + head] = (l_sum > 0.f) ? (m_used + log2f(l_sum)) / kLog2e : -INFINITY;
+            } else {
                 float* ml = part_ml + ((g * splits + sp) * kH + head) * 2;
-                ml[0] = (l_h > 0.f) ? m_h : -INFINITY;
-                ml[1] = l_h;
+                ml[0] = (l_sum > 0.f) ? m_used : -INFINITY;
+                ml[1] = l_sum;
             }
         }
     }
@@ -578,7 +592,7 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
     if (a.kv_dtype == LCS_F32) {
         const size_t smem = sizeof(float) * (a.H * a.D + kF32Chunk * a.D + a.H * kF32Chunk + a.H * a.d_v + 3 * a.H) +
                             sizeof(int) * (a.k > 0 ? a.k : 1);
-        cudaError_t e = cudaFuncSetAttribute(attend_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = set_smem_once(reinterpret_cast<const void*>(attend_f32_kernel), smem);
         if (e != cudaSuccess) return e;
         return launch_k(attend_f32_kernel, dim3((unsigned)queries), dim3(256), smem, s, pdl, a, status);
     }
@@ -594,7 +608,7 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
         part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256(queries * splits * kH * kDv * 4));
     }
     auto kern = (a.kv_dtype == LCS_KV_FP8) ? attend_tc_kernel<true> : attend_tc_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), kAtSmem);
     if (e != cudaSuccess) return e;
     e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, a, splits, part_o,
                  part_ml, status);

@@ -169,7 +169,7 @@ cudaError_t launch_t(const void* x, int64_t B, int64_t T, int d, const void* x_t
                      void* out, cudaStream_t s) {
     const size_t smem = sizeof(float) * kWarps * (((m + overlap + 3) & ~3) + d);
     auto kern = compress_kernel<Tin, Tout>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t err = set_smem_once(reinterpret_cast<const void*>(kern), smem);
     if (err != cudaSuccess) return err;
     const int64_t n = B * (T / m);
     if (n == 0) return cudaSuccess;

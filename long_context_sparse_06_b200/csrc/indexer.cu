@@ -238,7 +238,7 @@ cudaError_t launch_index_f32(const float* qI, const float* w, const float* kI, i
     const int64_t groups = B * Q;
     if (groups == 0 || N_c == 0) return cudaSuccess;
     const size_t smem = sizeof(float) * (H_I * d_I + H_I);
-    cudaError_t e = cudaFuncSetAttribute(index_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(index_f32_kernel), smem);
     if (e != cudaSuccess) return e;
     const int64_t ychunks = (N_c + 255) / 256;
     dim3 grid((unsigned)groups, (unsigned)(ychunks < 16 ? ychunks : 16));
@@ -260,7 +260,7 @@ cudaError_t launch_index_bf16_tc(const void* qI, const float* w, const void* kI,
                         kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     cudaError_t e =
-        cudaFuncSetAttribute(index_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIxSmem);
+        set_smem_once(reinterpret_cast<const void*>(index_bf16_tc_kernel), kIxSmem);
     if (e != cudaSuccess) return e;
     const int64_t total = groups * ((N_c + kBM - 1) / kBM);
     const int64_t grid = total < num_sms() ? total : num_sms();

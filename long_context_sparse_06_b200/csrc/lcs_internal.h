@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <utility>
+
 namespace lcs {
 
 // Workspace layout: [0, 256) status word; then the op's scratch regions, each
@@ -65,6 +68,10 @@ struct AttendArgs {
 };
 int64_t attend_scratch_bytes(const AttendArgs& a);
 cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaStream_t s, bool pdl);
+
+// Raises a kernel's dynamic shared-memory limit once per process and kernel (the
+// attribute call costs host time on every launch otherwise).
+cudaError_t set_smem_once(const void* kern, size_t bytes);
 
 // Launch helper with optional programmatic dependent launch.
 template <typename... KArgs, typename... Args>

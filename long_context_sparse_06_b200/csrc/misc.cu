@@ -149,7 +149,7 @@ cudaError_t launch_group_oproj(const float* o, int64_t T, int H, int d_v, const 
                                const float* Wo, int hidden, float* y, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     const size_t smem = sizeof(float) * (H * d_v + G * d_g);
-    cudaError_t err = cudaFuncSetAttribute(group_oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t err = set_smem_once(reinterpret_cast<const void*>(group_oproj_kernel), smem);
     if (err != cudaSuccess) return err;
     group_oproj_kernel<<<(unsigned)T, 256, smem, s>>>(o, H, d_v, Wg, G, d_g, Wo, hidden, y);
     return cudaGetLastError();

@@ -10,21 +10,25 @@
 // element is ranked by the 64-bit composite (key << 32 | ~index), so "larger
 // composite" is exactly "larger score, then lower index".
 //
-// One CTA of 1024 threads per query row, three coalesced passes over the row:
-//  1. Histogram of the top 14 bits of every key (sign, exponent and the top
-//     mantissa bits of the score) in shared memory; the bins are fine enough
-//     that the 32 lanes of a warp rarely collide on one counter.  A block-wide
-//     suffix scan finds the bin holding the k-th largest score: every key in a
-//     higher bin is selected, and `need` more come from the threshold bin.
-//  2. The threshold bin's elements are gathered in index order (each warp walks
-//     its own contiguous segment; slots from __ballot_sync / __popc) and ranked
-//     exactly by counting, on the composite key.
-//  3. Ordered compaction: each warp re-walks its segment and writes the selected
-//     indices at offsets from ballots, so the output is ascending without a sort.
-// If the threshold bin is too crowded for the counting rank (massive ties) the
-// row falls back to an exact MSB-first radix select (8-bit digits, shared-memory
-// histograms) followed by the same kind of ordered compaction.  The result does
-// not depend on the order of the shared atomics, so every step is deterministic.
+// One CTA of 512 threads per query row:
+//  1. Lower bound: a fixed strided sample of 512 keys is histogrammed over the
+//     top 14 key bits (sign, exponent, top mantissa bits); the lower edge of the
+//     bin holding the sample's rank-r element, r about 1.5 k x sample/row + 8,
+//     bounds the k-th score from below with overwhelming probability.
+//  2. One pass over the row: each lane loads 32 consecutive keys with 16-byte
+//     vector loads and appends those >= the bound to its warp's buffer; slots
+//     come from per-lane counts and a warp scan, so candidates stay in index
+//     order.
+//  3. The candidates (about 1.5 k) are histogrammed on the same 14 bits; a
+//     suffix scan finds the bin holding the k-th largest; that bin's members are
+//     ranked exactly by counting on the composite key; an ordered compaction over
+//     the candidate list (warp slices, __ballot_sync / __popc for the slots) writes
+//     the ascending selection.
+// Shared-memory atomics: ~1024 + ~1.5 k per row instead of one per entry.  If
+// the bound misses (fewer than k candidates, a full buffer, a crowded bin) the
+// row falls back to an exact MSB-first radix select (8-bit digits) followed by
+// an ordered ballot compaction.  Nothing depends on the order of the atomics,
+// so every step is deterministic.
 #include <utility>
 
 #include "lcs_common.cuh"
@@ -34,23 +38,29 @@ namespace lcs {
 
 namespace {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBinBits = 14;
 constexpr int kBins = 1 << kBinBits;
 constexpr int kCandCap = 2048;                 // threshold-bin elements ranked by counting
-constexpr int kWarpCap = 256;                  // per-warp gather buffer
+constexpr int kWarpCap = 512;                  // per-warp candidate buffer
+constexpr int kListCap = kWarps * kWarpCap;    // all candidates
 
 struct TopkSmem {
-    uint32_t bins[kBins];                       // 64 KB histogram
-    unsigned long long wbuf[kWarps * kWarpCap]; // per-warp gather buffers (64 KB)
-    unsigned long long cand[kCandCap];          // threshold-bin candidates in index order
-    uint8_t take[kCandCap];                     // candidate selected?
+    uint32_t bins[kBins + kBins / 32];          // 64 KB histogram, one pad word per 32 bins
+    unsigned long long wbuf[kListCap];          // per-warp candidate buffers (64 KB)
+    unsigned long long list[kListCap];          // compacted candidates, index order (64 KB)
+    uint8_t take[kListCap];                     // candidate selected?
+    uint16_t mpos[kCandCap];                    // list positions of the threshold bin's members
     uint32_t hist[256], scan[256];              // radix fallback
     uint32_t warp_cnt[kWarps], warp_off[kWarps], warp_gt[kWarps], warp_sel[kWarps];
     uint32_t wsum[kWarps];
-    uint32_t digit, krem, tbin, above, fail;
+    uint32_t digit, krem, tbin, above, fail, total;
 };
+
+// Histogram slot of bin b: one pad word after every 32 bins, so that threads owning
+// 32 consecutive bins read different banks.
+__device__ __forceinline__ uint32_t hb(uint32_t b) { return b + (b >> 5); }
 
 template <bool BF16>
 __device__ __forceinline__ uint32_t load_key(const void* row, int64_t i) {
@@ -129,7 +139,88 @@ __device__ void radix_select(TopkSmem& sm, const void* srow, int64_t n, int k, i
     }
 }
 
-// ------------------------------------------------------------------ kernel
+// Exclusive prefix over the kWarps per-warp values in sm.wsum (scanned in place by
+// warp 0; lanes >= kWarps carry zeros and write nothing).
+static_assert(kWarps <= 32, "one warp scans the per-warp sums");
+__device__ __forceinline__ void scan_warp_sums(TopkSmem& sm) {
+    if (threadIdx.x < 32) {
+        const uint32_t v = (threadIdx.x < kWarps) ? sm.wsum[threadIdx.x] : 0u;
+        uint32_t incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+            if (threadIdx.x >= o) incl += x;
+        }
+        if (threadIdx.x < kWarps) sm.wsum[threadIdx.x] = incl - v;
+        if (threadIdx.x == kWarps - 1) sm.total = incl;
+    }
+    __syncthreads();
+}
+
+// Block-wide: the bin holding the k-th largest of the histogram (bins in descending
+// order of value from the top).  Sets sm.tbin and sm.above (count in higher bins).
+__device__ void find_bin(TopkSmem& sm, uint32_t k) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    constexpr int kPer = kBins / kThreads;      // thread 0 owns the top bins
+    const int hi_bin = kBins - 1 - t * kPer;
+    uint32_t c[kPer];
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) { c[j] = sm.bins[hb(hi_bin - j)]; local += c[j]; }
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) sm.wsum[warp] = incl;
+    __syncthreads();
+    scan_warp_sums(sm);
+    const uint32_t excl = sm.wsum[warp] + incl - local;
+    if (excl < k && excl + local >= k) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            if (run + c[j] >= k) { sm.tbin = hi_bin - j; sm.above = run; break; }
+            run += c[j];
+        }
+    }
+    __syncthreads();
+}
+
+// Loads the 32 consecutive keys [i0, i0+32) of lane-owned scores (clipped at n).
+template <bool BF16>
+__device__ __forceinline__ void load32(const char* srow, int64_t i0, int64_t n, uint32_t (&key)[32]) {
+    if (i0 + 32 <= n) {
+        if constexpr (BF16) {
+            const uint4* p = reinterpret_cast<const uint4*>(srow + i0 * 2);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint4 w = __ldg(p + v);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    key[8 * v + 2 * q] = bf16_key((uint16_t)(ww[q] & 0xFFFF));
+                    key[8 * v + 2 * q + 1] = bf16_key((uint16_t)(ww[q] >> 16));
+                }
+            }
+        } else {
+            const float4* p = reinterpret_cast<const float4*>(srow + i0 * 4);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const float4 f = __ldg(p + v);
+                key[4 * v] = f32_key(f.x);
+                key[4 * v + 1] = f32_key(f.y);
+                key[4 * v + 2] = f32_key(f.z);
+                key[4 * v + 3] = f32_key(f.w);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) key[j] = (i0 + j < n) ? load_key<BF16>(srow, i0 + j) : 0u;
+    }
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restrict__ scores, int64_t N_c,
                                                            const int64_t* __restrict__ q_pos, int m, int k,
@@ -156,69 +247,55 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
         return;
     }
 
-    // ---- 1. histogram of the top bits, then the threshold bin by a suffix scan
-    for (int i = t; i < kBins; i += kThreads) sm.bins[i] = 0;
+    // ---- 1. lower bound from a strided sample of one key per thread
+    for (int i = t; i < kBins + kBins / 32; i += kThreads) sm.bins[i] = 0;
     __syncthreads();
-    for (int64_t i = t; i < n; i += kThreads) atomicAdd(&sm.bins[load_key<BF16>(srow, i) >> kShift], 1u);
-    __syncthreads();
-    constexpr int kPer = kBins / kThreads;      // bins per thread, thread 0 owns the top ones
-    const int hi_bin = kBins - 1 - t * kPer;
-    uint32_t local = 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) local += sm.bins[hi_bin - j];
-    uint32_t incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+    uint32_t T = 0;
+    if (n > kListCap / 2) {
+        atomicAdd(&sm.bins[hb(load_key<BF16>(srow, (int64_t)(((uint64_t)t * (uint64_t)n) / kThreads)) >> kShift)], 1u);
+        __syncthreads();
+        uint32_t r = (uint32_t)((3 * (int64_t)k * kThreads) / (2 * n)) + 8;
+        if (r > (uint32_t)kThreads) r = kThreads;
+        find_bin(sm, r);
+        T = sm.tbin << kShift;
+        for (int i = t; i < kBins + kBins / 32; i += kThreads) sm.bins[i] = 0;
     }
-    if (lane == 31) sm.wsum[warp] = incl;
-    __syncthreads();
-    uint32_t wbase = 0;
-    for (int w = 0; w < warp; ++w) wbase += sm.wsum[w];
-    const uint32_t excl = wbase + incl - local;
-    if (excl < (uint32_t)k && excl + local >= (uint32_t)k) {
-        uint32_t run = excl;
-        for (int j = 0; j < kPer; ++j) {
-            const uint32_t c = sm.bins[hi_bin - j];
-            if (run + c >= (uint32_t)k) { sm.tbin = hi_bin - j; sm.above = run; break; }
-            run += c;
-        }
-    }
-    __syncthreads();
-    const uint32_t tbin = sm.tbin, above = sm.above, need = (uint32_t)k - above;
-    const uint32_t m_t = sm.bins[tbin];          // elements in the threshold bin
 
-    // ---- 2. gather the threshold bin in index order; count the keys above it
-    const int64_t seg = ((n + kWarps - 1) / kWarps + 31) / 32 * 32;
-    const int64_t s0 = warp * seg, s1 = (s0 + seg < n) ? s0 + seg : n;
-    const uint32_t lt = (1u << lane) - 1u;
+    // ---- 2. one pass: lane-owned runs of 32 consecutive keys; keys >= T go to the warp's
+    // buffer in index order (per-lane counts, warp scan for the lane's slot base)
     unsigned long long* wb = sm.wbuf + warp * kWarpCap;
-    uint32_t cnt = 0, gt = 0;
-    if (m_t <= kCandCap) {
-        for (int64_t base = s0; base < s1; base += 32) {
-            const int64_t i = base + lane;
-            const bool act = i < s1;
-            const uint32_t key = act ? load_key<BF16>(srow, i) : 0u;
-            const uint32_t bn = key >> kShift;
-            const bool eq = act && bn == tbin;
-            const uint32_t em = __ballot_sync(0xffffffffu, eq);
-            const uint32_t slot = cnt + __popc(em & lt);
-            if (eq && slot < kWarpCap)
-                wb[slot] = ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)i);
-            cnt += __popc(em);
-            gt += __popc(__ballot_sync(0xffffffffu, act && bn > tbin));
+    const int64_t per_warp = ((n + kWarps - 1) / kWarps + 1023) / 1024 * 1024;   // whole 32x32 batches
+    const int64_t w0 = warp * per_warp, w1 = (w0 + per_warp < n) ? w0 + per_warp : n;
+    uint32_t wcnt = 0;
+    for (int64_t bb = w0; bb < w1; bb += 1024) {
+        const int64_t i0 = bb + 32 * lane;
+        uint32_t key[32];
+        load32<BF16>(srow, i0, w1, key);
+        uint32_t c = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) c += (i0 + j < w1 && key[j] >= T);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += x;
         }
+        uint32_t slot = wcnt + incl - c;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (i0 + j < w1 && key[j] >= T) {
+                if (slot < kWarpCap)
+                    wb[slot] = ((unsigned long long)key[j] << 32) | (unsigned long long)(~(uint32_t)(i0 + j));
+                ++slot;
+            }
+        wcnt += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) { sm.warp_cnt[warp] = cnt; sm.warp_gt[warp] = gt; }
+    if (lane == 0) { sm.warp_cnt[warp] = wcnt; sm.wsum[warp] = wcnt; }
     __syncthreads();
+    scan_warp_sums(sm);
     if (t == 0) {
-        uint32_t off = 0, fail = m_t > kCandCap;
-        for (int w = 0; w < kWarps; ++w) {
-            sm.warp_off[w] = off;
-            off += sm.warp_cnt[w];
-            fail |= sm.warp_cnt[w] > (uint32_t)kWarpCap;
-        }
+        uint32_t fail = sm.total < (uint32_t)k;
+        for (int w = 0; w < kWarps; ++w) fail |= sm.warp_cnt[w] > (uint32_t)kWarpCap;
         sm.fail = fail;
     }
     __syncthreads();
@@ -226,43 +303,74 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
         radix_select<BF16>(sm, srow, n, k, out);
         return;
     }
-    for (uint32_t j = lane; j < cnt; j += 32) sm.cand[sm.warp_off[warp] + j] = wb[j];
+    const uint32_t C = sm.total;
+    {
+        const uint32_t o = sm.wsum[warp];
+        for (uint32_t j = lane; j < wcnt; j += 32) sm.list[o + j] = wb[j];
+    }
     __syncthreads();
 
-    // ---- rank the threshold bin by counting (composite keys are distinct)
+    // ---- 3. exact selection among the candidates
+    for (uint32_t j = t; j < C; j += kThreads) atomicAdd(&sm.bins[hb((uint32_t)(sm.list[j] >> 32) >> kShift)], 1u);
+    __syncthreads();
+    find_bin(sm, (uint32_t)k);
+    const uint32_t tbin = sm.tbin, need = (uint32_t)k - sm.above;
+    const uint32_t m_t = sm.bins[hb(tbin)];
+    if (m_t > kCandCap) {
+        radix_select<BF16>(sm, srow, n, k, out);
+        return;
+    }
+    // The list is split into 32 contiguous slices, one per warp, walked in tiles of 32.
+    const uint32_t slice = (C + kWarps - 1) / kWarps;
+    const uint32_t l0 = warp * slice, l1 = (l0 + slice < C) ? l0 + slice : C;
+    const uint32_t lt = (1u << lane) - 1u;
+    // threshold-bin members: count per slice, then compact in list order
+    uint32_t mc = 0;
+    for (uint32_t bs = l0; bs < l1; bs += 32) {
+        const uint32_t j = bs + lane;
+        const bool mem = j < l1 && ((uint32_t)(sm.list[j] >> 32) >> kShift) == tbin;
+        mc += __popc(__ballot_sync(0xffffffffu, mem));
+    }
+    if (lane == 0) sm.wsum[warp] = mc;
+    __syncthreads();
+    scan_warp_sums(sm);
+    {
+        uint32_t pos = sm.wsum[warp];
+        for (uint32_t bs = l0; bs < l1; bs += 32) {
+            const uint32_t j = bs + lane;
+            const uint32_t bn = j < l1 ? ((uint32_t)(sm.list[j] >> 32) >> kShift) : 0u;
+            const bool mem = j < l1 && bn == tbin;
+            const uint32_t mm = __ballot_sync(0xffffffffu, mem);
+            if (mem) sm.mpos[pos + __popc(mm & lt)] = (uint16_t)j;
+            if (j < l1) sm.take[j] = bn > tbin;
+            pos += __popc(mm);
+        }
+    }
+    __syncthreads();
+    // rank the members among themselves by counting (composite keys are distinct)
     for (uint32_t j = t; j < m_t; j += kThreads) {
-        const unsigned long long c = sm.cand[j];
+        const unsigned long long c = sm.list[sm.mpos[j]];
         uint32_t r = 0;
-        for (uint32_t i = 0; i < m_t; ++i) r += sm.cand[i] > c;
-        sm.take[j] = r < need;
+        for (uint32_t i = 0; i < m_t; ++i) r += sm.list[sm.mpos[i]] > c;
+        sm.take[sm.mpos[j]] = r < need;
     }
     __syncthreads();
-    {   // selected candidates per warp segment
-        const uint32_t o = sm.warp_off[warp];
-        uint32_t c = 0;
-        for (uint32_t j = lane; j < cnt; j += 32) c += sm.take[o + j];
-#pragma unroll
-        for (int x = 16; x > 0; x >>= 1) c += __shfl_xor_sync(0xffffffffu, c, x);
-        if (lane == 0) sm.warp_sel[warp] = c;
+    // ordered compaction over the candidate list (already in index order)
+    uint32_t sc = 0;
+    for (uint32_t bs = l0; bs < l1; bs += 32) {
+        const uint32_t j = bs + lane;
+        sc += __popc(__ballot_sync(0xffffffffu, j < l1 && sm.take[j]));
     }
+    if (lane == 0) sm.wsum[warp] = sc;
     __syncthreads();
-
-    // ---- 3. ordered compaction
-    uint32_t pos = 0;
-    for (int w = 0; w < warp; ++w) pos += sm.warp_gt[w] + sm.warp_sel[w];
-    uint32_t ci = sm.warp_off[warp];
-    for (int64_t base = s0; base < s1; base += 32) {
-        const int64_t i = base + lane;
-        const bool act = i < s1;
-        const uint32_t key = act ? load_key<BF16>(srow, i) : 0u;
-        const uint32_t bn = key >> kShift;
-        const bool eq = act && bn == tbin;
-        const uint32_t em = __ballot_sync(0xffffffffu, eq);
-        const bool tk = (act && bn > tbin) || (eq && sm.take[ci + __popc(em & lt)]);
+    scan_warp_sums(sm);
+    uint32_t pos = sm.wsum[warp];
+    for (uint32_t bs = l0; bs < l1; bs += 32) {
+        const uint32_t j = bs + lane;
+        const bool tk = j < l1 && sm.take[j];
         const uint32_t tm = __ballot_sync(0xffffffffu, tk);
-        if (tk) out[pos + __popc(tm & lt)] = (int32_t)i;
+        if (tk) out[pos + __popc(tm & lt)] = (int32_t)(~(uint32_t)(sm.list[j] & 0xFFFFFFFFull));
         pos += __popc(tm);
-        ci += __popc(em);
     }
 }
 
@@ -283,12 +391,12 @@ cudaError_t launch_topk(const void* scores, int score_dtype, int64_t B, int64_t 
     if (rows == 0 || k == 0) return cudaSuccess;
     const size_t smem = sizeof(TopkSmem);
     if (score_dtype == LCS_BF16) {
-        cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = set_smem_once(reinterpret_cast<const void*>(topk_kernel<true>), smem);
         if (e != cudaSuccess) return e;
         return launch_k(topk_kernel<true>, dim3((unsigned)rows), dim3(kThreads), smem, s, pdl, scores, N_c, q_pos, m,
                         k, idx);
     }
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(topk_kernel<false>), smem);
     if (e != cudaSuccess) return e;
     return launch_k(topk_kernel<false>, dim3((unsigned)rows), dim3(kThreads), smem, s, pdl, scores, N_c, q_pos, m, k,
                     idx);
