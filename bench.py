@@ -1,19 +1,28 @@
 #!/usr/bin/env python3
-"""Benchmark of the CSA decode step (the hot path of the compressed sparse attention).
+"""Benchmark of the CSA / HCA compressed-attention hot path on B200.
 
-Workload (one attention layer, one decode step = one new token for each of B
-requests): CSA decode, bf16 -- 32 requests with a 128K-token context each:
-32768 compressed entries (m = 4) of dim 576 (512 content + 64 RoPE), 64 query
-heads sharing the KV, lightning indexer with 64 heads x 128 dims over bf16 keys,
-top-512 selection, a 128-row raw window; values N(0,1), query scale 1/sqrt(576).
-A step runs the whole path (index scoring -> top-k -> sparse MQA) through
-decode_fused.
+Default workload (the headline): CSA decode, bf16 -- 32 requests with a 128K-token
+context each: 32768 compressed entries (m = 4) of dim 576 (512 content + 64 RoPE),
+64 query heads sharing the KV, lightning indexer 64 heads x 128 over bf16 keys,
+top-512, a 128-row raw window; N(0,1) values, query scale 1/sqrt(576).  One step
+= one decode token for every request = index scoring -> top-k -> sparse MQA
+(decode_fused), captured once as a CUDA graph and replayed.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Other workloads (`--workload`) measure the remaining rows of the path:
+  hca_decode_bf16_1m     16 requests x 8192 entries (1M tokens, m' = 128), dense MQA
+  csa_decode_mixed_1m    4 requests x 262144 entries, FP8 KV + bf16 RoPE dims,
+                         FP4 index keys, bf16 scores, top-1024
+  csa_prefill_bf16_8k    8192 new tokens after a 131072-token prefix: compress the
+                         chunk's KV and index keys, causal index + top-1024, attention
+  compress_stream_1m     1M raw rows x 576 bf16: CSA (m=4, overlap 2) and HCA
+                         (m'=128) compression of the KV, CSA of 128-dim index keys
 
-N > 1 is launched with torchrun: every rank runs its own batch of 32 requests on
-its own GPU (requests are independent: no collective on the data path); the
-step time is the max over ranks.  One JSON line is printed by rank 0.
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+  python bench.py --stage index|topk|attend|compress ...   (one stage alone, for ncu)
+
+N > 1 is launched with torchrun: every rank runs its own copy of the workload on
+its own GPU (requests are independent: no collective on the data path); the step
+time is the max over ranks.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -23,7 +32,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -32,24 +40,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "CSA/HCA decode tok/s and achieved HBM GB/s vs roofline at 128K-1M ctx"
-UNIT = "tok/s"
-WORKLOAD = dict(workload="csa_decode_bf16_128k", requests=32, context_tokens=131072, compressed_entries=32768,
-                m=4, kv_dim=576, d_v=512, heads=64, index_heads=64, index_dim=128, topk=512, window=128)
-B, NC, D, DV, H, HI, DI, K, TW = 32, 32768, 576, 512, 64, 64, 128, 512, 128
+D, DV, H, HI, DI, TW = 576, 512, 64, 64, 128, 128
 SCALE = 1.0 / math.sqrt(576.0)
-
-
-def algorithmic_bytes_per_request():
-    keys = NC * DI * 2
-    sel = K * D * 2
-    win = TW * D * 2
-    qin = H * D * 2 + HI * DI * 2 + HI * 4
-    out = H * DV * 2
-    return keys + sel + win + qin + out
-
-
-def index_bytes_per_request():
-    return NC * DI * 2 + HI * DI * 2 + HI * 4
 
 
 def load_peaks():
@@ -57,8 +49,8 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 def kernel_source_hash(files):
@@ -69,17 +61,26 @@ def kernel_source_hash(files):
     return h.hexdigest()[:16]
 
 
-INDEX_KERNEL_FILES = ["long_context_sparse_06_b200/csrc/indexer.cu", "long_context_sparse_06_b200/csrc/lcs_common.cuh"]
+KERNEL_FILES = {
+    "index_bf16_tc_kernel": ["long_context_sparse_06_b200/csrc/indexer.cu",
+                             "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
+    "index_fp4_tc_kernel": ["long_context_sparse_06_b200/csrc/indexer_fp4.cu",
+                            "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
+    "attend_tc_kernel": ["long_context_sparse_06_b200/csrc/attend.cu",
+                         "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
+    "compress_kernel": ["long_context_sparse_06_b200/csrc/compress.cu",
+                        "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
+}
 
 
-def recorded_traffic(kernel):
+def recorded_traffic(kernel, workload):
     """dram bytes per launch from a committed ncu summary, if taken on the current source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f).get(kernel)
-    if not d or d.get("source_hash") != kernel_source_hash(INDEX_KERNEL_FILES):
+        d = json.load(f).get(f"{kernel}@{workload}")
+    if not d or d.get("source_hash") != kernel_source_hash(KERNEL_FILES[kernel]):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -89,7 +90,7 @@ class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while the timed region runs."""
 
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
-               0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+               0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, device_index):
         self.samples, self.reasons, self.max_mhz = [], set(), None
@@ -99,11 +100,12 @@ class ClockSampler:
             import pynvml
             import torch
             pynvml.nvmlInit()
-            bus = torch.cuda.get_device_properties(device_index)
-            pci = getattr(bus, "pci_bus_id", None)
+            props = torch.cuda.get_device_properties(device_index)
+            pci = getattr(props, "pci_bus_id", None)
             if pci is not None:
-                dom = getattr(bus, "pci_domain_id", 0)
-                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{pci:02x}:{getattr(bus, 'pci_device_id', 0):02x}.0")
+                dom = getattr(props, "pci_domain_id", 0)
+                dev_id = getattr(props, "pci_device_id", 0)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{pci:02x}:{dev_id:02x}.0")
             else:
                 vis = os.environ.get("CUDA_VISIBLE_DEVICES")
                 idx = int(vis.split(",")[device_index]) if vis else device_index
@@ -118,7 +120,7 @@ class ClockSampler:
         self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
         r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
         for bit, name in self.REASONS.items():
-            if r & bit and name != "gpu_idle":
+            if r & bit:
                 self.reasons.add(name)
 
     def _run(self):
@@ -127,7 +129,7 @@ class ClockSampler:
                 self._sample()
             except Exception:
                 pass
-            self._stop.wait(0.01)
+            self._stop.wait(0.005)
 
     def __enter__(self):
         if self._h is not None:
@@ -147,24 +149,413 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-# ------------------------------------------------------------------ inputs
-def make_inputs(device, rank):
-    import torch
-    from long_context_sparse_06_b200 import synth
-    tag = f"bench.r{rank}."
-    bf = torch.bfloat16
-    x = dict(
-        q=synth.normal_t(tag + "q", (B, H, D), dtype=bf, device=device),
-        comp=synth.normal_t(tag + "comp", (B, NC, D), dtype=bf, device=device),
-        win=synth.normal_t(tag + "win", (B, TW, D), dtype=bf, device=device),
-        qI=synth.normal_t(tag + "qI", (B, HI, DI), dtype=bf, device=device),
-        w=synth.normal_t(tag + "w", (B, HI), std=1.0 / 8, dtype=torch.float32, device=device),
-        kI=synth.normal_t(tag + "kI", (B, NC, DI), dtype=bf, device=device),
-    )
-    return x
+# --------------------------------------------------------------- workloads
+class Workload:
+    """One configuration of the path: inputs, the step, stages and accounting."""
+    name = ""
+    unit = "tok/s"
+    bound = "hbm"
+    stage_names = ()
+
+    def __init__(self, lcs, dev, rank):
+        self.lcs, self.dev, self.rank = lcs, dev, rank
+
+    def tag(self, s):
+        return f"bench.{self.name}.r{self.rank}.{s}"
+
+    def dominant_stage(self):
+        return 0
 
 
-# ------------------------------------------------------------------- arms
+class CsaDecode(Workload):
+    """CSA decode: decode_fused(MODE_CSA) over B requests."""
+    name = "csa_decode_bf16_128k"
+    B, NC, K = 32, 32768, 512
+    mixed = False
+    stage_names = ("index", "topk", "attend")
+    dominant = "index_bf16_tc_kernel"
+
+    def config(self):
+        return dict(workload=self.name, requests=self.B, context_tokens=self.NC * 4, compressed_entries=self.NC, m=4,
+                    kv_dim=D, d_v=DV, heads=H, index_heads=HI, index_dim=DI, topk=self.K, window=TW,
+                    kv_format="fp8-e4m3 (pow2 scale per 128) + bf16 rope" if self.mixed else "bf16",
+                    index_key_format="fp4-e2m1 + e4m3 scale per 32" if self.mixed else "bf16",
+                    score_format="bf16" if self.mixed else "fp32")
+
+    def build(self):
+        import torch
+        from long_context_sparse_06_b200 import synth
+        L, dev, bf = self.lcs, self.dev, torch.bfloat16
+        B, NC = self.B, self.NC
+        self.q = synth.normal_t(self.tag("q"), (B, H, D), dtype=bf, device=dev)
+        self.qI = synth.normal_t(self.tag("qI"), (B, HI, DI), dtype=bf, device=dev)
+        self.w = synth.normal_t(self.tag("w"), (B, HI), std=1.0 / 8, device=dev)
+        if self.mixed:
+            f32 = torch.float32
+            comp = synth.with_outliers_t(self.tag("comp"), synth.normal_t(self.tag("comp"), (B, NC, D), dtype=f32,
+                                                                            device=dev))
+            self.comp = L.lcs_quant_kv_fp8(comp)
+            del comp
+            win = synth.with_outliers_t(self.tag("win"), synth.normal_t(self.tag("win"), (B, TW, D), dtype=f32,
+                                                                          device=dev))
+            self.win = L.lcs_quant_kv_fp8(win)
+            kraw = synth.with_outliers_t(self.tag("kI"), synth.normal_t(self.tag("kI"), (B, NC, DI), dtype=f32,
+                                                                          device=dev))
+            self.kI = L.lcs_quant_fp4(kraw)
+            del kraw
+            self.kv_dtype, self.kI_dtype, self.score_dtype, self.row = L.KV_FP8, L.FP4, L.BF16, 656
+        else:
+            self.comp = synth.normal_t(self.tag("comp"), (B, NC, D), dtype=bf, device=dev)
+            self.win = synth.normal_t(self.tag("win"), (B, TW, D), dtype=bf, device=dev)
+            self.kI = synth.normal_t(self.tag("kI"), (B, NC, DI), dtype=bf, device=dev)
+            self.kv_dtype, self.kI_dtype, self.score_dtype, self.row = L.BF16, L.BF16, L.F32, 2 * D
+        self.out = torch.empty((B, H, DV), dtype=bf, device=dev)
+        self.ws = L.workspace(L.lcs_workspace_size(L.OP_DECODE, B, 1, NC, TW, self.K, H, DV, self.score_dtype), dev)
+        torch.cuda.synchronize()
+
+    def step(self, stream):
+        L = self.lcs
+        L.decode_fused(L.MODE_CSA, self.q, self.comp, self.win, DV, SCALE, kv_dtype=self.kv_dtype, qI=self.qI,
+                       w=self.w, kI=self.kI, kI_dtype=self.kI_dtype, k=self.K, score_dtype=self.score_dtype,
+                       out=self.out, ws=self.ws, stream=stream)
+
+    def stage(self, name, stream):
+        """One stage alone (for profiling); index and top-k run as csa_index_topk."""
+        L = self.lcs
+        if name in ("index", "topk"):
+            L.csa_index_topk(self.qI.view(self.B, 1, HI, DI), self.w.view(self.B, 1, HI), self.kI, self.K,
+                             N_c=self.NC, kI_dtype=self.kI_dtype, score_dtype=self.score_dtype, stream=stream)
+        elif name == "attend":
+            if not hasattr(self, "idx"):
+                import torch
+                self.idx = L.csa_index_topk(self.qI.view(self.B, 1, HI, DI), self.w.view(self.B, 1, HI), self.kI,
+                                            self.K, N_c=self.NC, kI_dtype=self.kI_dtype,
+                                            score_dtype=self.score_dtype).contiguous()
+                torch.cuda.synchronize()
+            L.csa_attend(self.q.view(self.B, 1, H, D), self.comp, self.win, self.idx, DV, SCALE,
+                         kv_dtype=self.kv_dtype, stream=stream)
+
+    def units_per_step(self):
+        return self.B
+
+    def key_bytes(self):
+        return self.NC * (DI // 2 + DI // 32 if self.mixed else DI * 2)
+
+    def alg_bytes_per_step(self):
+        rows = (self.K + TW) * self.row
+        qin = H * D * 2 + HI * DI * 2 + HI * 4
+        return self.B * (self.key_bytes() + rows + qin + H * DV * 2)
+
+    def dominant_bytes(self):
+        return self.B * (self.key_bytes() + HI * DI * 2 + HI * 4)
+
+    def e2e_io(self):
+        """Every per-step input (device tensors) and the step's result."""
+        return [self.q, self.qI, self.w], self.out
+
+    def cpu_sample(self, budget_s):
+        """The oracle on whole requests of this workload until about budget_s seconds."""
+        import numpy as np
+        from oracle import oracle as orc
+        el, n = 0.0, 0
+        if self.mixed:
+            planes = self.kI.cpu().numpy()
+            tot = self.B * self.NC
+        while n < self.B and el < budget_s:
+            q = self.q[n].double().cpu().numpy()
+            qI = self.qI[n].double().cpu().numpy()
+            w = self.w[n].cpu().numpy()
+            if self.mixed:
+                kp = planes[:tot * 64].reshape(self.B, self.NC, 64)[n]
+                ks = planes[tot * 64:].reshape(self.B, self.NC, 4)[n]
+                comp_rows = self.comp[n].cpu().numpy()
+                win_rows = self.win[n].cpu().numpy()
+                qf = self.qI[n].float().cpu().numpy()
+                ts = time.perf_counter()
+                s = orc.index_scores_fp4(qf, w, kp, ks).astype(np.float32)
+                idx = orc.topk(s, self.K)
+                comp = orc.dequant_kv_fp8(comp_rows)
+                win = orc.dequant_kv_fp8(win_rows)
+            else:
+                kI = self.kI[n].double().cpu().numpy()
+                comp = self.comp[n].double().cpu().numpy()
+                win = self.win[n].double().cpu().numpy()
+                ts = time.perf_counter()
+                s = orc.index_scores_bf16(qI, w, kI)
+                idx = orc.topk(s, self.K)
+            orc.csa_attend(q, comp, idx, win, 0, -1, TW, DV, SCALE)
+            el += time.perf_counter() - ts
+            n += 1
+        return n, el, f"{n} of {self.B} requests, full path per request (index over all {self.NC} entries, " \
+                      f"top-{self.K}, attention over {self.K}+{TW} rows); single thread"
+
+
+class CsaDecodeMixed(CsaDecode):
+    name = "csa_decode_mixed_1m"
+    B, NC, K = 4, 262144, 1024
+    mixed = True
+    dominant = "index_fp4_tc_kernel"
+
+
+class HcaDecode(Workload):
+    name = "hca_decode_bf16_1m"
+    B, NC = 16, 8192
+    stage_names = ("attend",)
+    dominant = "attend_tc_kernel"
+
+    def config(self):
+        return dict(workload=self.name, requests=self.B, context_tokens=self.NC * 128, compressed_entries=self.NC,
+                    m=128, kv_dim=D, d_v=DV, heads=H, window=TW, kv_format="bf16")
+
+    def build(self):
+        import torch
+        from long_context_sparse_06_b200 import synth
+        L, dev, bf = self.lcs, self.dev, torch.bfloat16
+        self.q = synth.normal_t(self.tag("q"), (self.B, H, D), dtype=bf, device=dev)
+        self.comp = synth.normal_t(self.tag("comp"), (self.B, self.NC, D), dtype=bf, device=dev)
+        self.win = synth.normal_t(self.tag("win"), (self.B, TW, D), dtype=bf, device=dev)
+        self.out = torch.empty((self.B, H, DV), dtype=bf, device=dev)
+        self.ws = L.workspace(L.lcs_workspace_size(L.OP_DECODE, self.B, 1, self.NC, TW, 0, H, DV), dev)
+
+    def step(self, stream):
+        L = self.lcs
+        L.decode_fused(L.MODE_HCA, self.q, self.comp, self.win, DV, SCALE, out=self.out, ws=self.ws, stream=stream)
+
+    def stage(self, name, stream):
+        self.step(stream)
+
+    def units_per_step(self):
+        return self.B
+
+    def alg_bytes_per_step(self):
+        return self.B * ((self.NC + TW) * D * 2 + H * D * 2 + H * DV * 2)
+
+    def dominant_bytes(self):
+        return self.alg_bytes_per_step()
+
+    def e2e_io(self):
+        return [self.q], self.out
+
+    def cpu_sample(self, budget_s):
+        from oracle import oracle as orc
+        el, n = 0.0, 0
+        while n < self.B and el < budget_s:
+            q = self.q[n].double().cpu().numpy()
+            comp = self.comp[n].double().cpu().numpy()
+            win = self.win[n].double().cpu().numpy()
+            ts = time.perf_counter()
+            orc.hca_attend(q, comp, 128, win, 0, -1, TW, DV, SCALE)
+            el += time.perf_counter() - ts
+            n += 1
+        return n, el, f"{n} of {self.B} requests, dense attention over {self.NC}+{TW} rows each; single thread"
+
+
+class CsaPrefill(Workload):
+    """Chunked prefill: 8192 new tokens after a 131072-token prefix."""
+    name = "csa_prefill_bf16_8k"
+    unit = "query-tok/s"
+    bound = "tensor"
+    P0, Q, K = 131072, 8192, 1024
+    stage_names = ("compress", "index", "topk", "attend")
+    dominant = "index_bf16_tc_kernel"
+
+    def config(self):
+        return dict(workload=self.name, requests=1, prefix_tokens=self.P0, new_tokens=self.Q, m=4, overlap=2,
+                    compressed_entries=(self.P0 + self.Q) // 4, kv_dim=D, d_v=DV, heads=H, index_heads=HI,
+                    index_dim=DI, topk=self.K, window=TW, kv_format="bf16", causal=True)
+
+    def build(self):
+        import torch
+        from long_context_sparse_06_b200 import synth
+        L, dev, bf = self.lcs, self.dev, torch.bfloat16
+        Q, P0 = self.Q, self.P0
+        self.NC = (P0 + Q) // 4
+        n0 = P0 // 4
+        self.comp = torch.empty((1, self.NC, D), dtype=bf, device=dev)
+        self.comp[:, :n0] = synth.normal_t(self.tag("prefix_comp"), (1, n0, D), dtype=bf, device=dev)
+        self.kI = torch.empty((1, self.NC, DI), dtype=bf, device=dev)
+        self.kI[:, :n0] = synth.normal_t(self.tag("prefix_kI"), (1, n0, DI), dtype=bf, device=dev)
+        self.x = synth.normal_t(self.tag("x"), (1, Q, D), dtype=bf, device=dev)           # raw chunk KV
+        self.x_tail = synth.normal_t(self.tag("x_tail"), (1, 2, D), dtype=bf, device=dev)
+        self.kx = synth.normal_t(self.tag("kx"), (1, Q, DI), dtype=bf, device=dev)        # raw index keys
+        self.kx_tail = synth.normal_t(self.tag("kx_tail"), (1, 2, DI), dtype=bf, device=dev)
+        self.z = synth.normal_t(self.tag("z"), (1, Q), device=dev)
+        self.z_tail = synth.normal_t(self.tag("z_tail"), (1, 2), device=dev)
+        self.zI = synth.normal_t(self.tag("zI"), (1, Q), device=dev)
+        self.zI_tail = synth.normal_t(self.tag("zI_tail"), (1, 2), device=dev)
+        self.bias = synth.normal_t(self.tag("bias"), (6,), device=dev)
+        self.biasI = synth.normal_t(self.tag("biasI"), (6,), device=dev)
+        self.win = synth.normal_t(self.tag("win"), (1, 127 + Q, D), dtype=bf, device=dev)  # post-RoPE rows
+        self.win_pos0 = torch.tensor([P0 - 127], dtype=torch.int64, device=dev)
+        self.q_pos = (P0 + torch.arange(Q, dtype=torch.int64, device=dev)).view(1, Q)
+        self.q = synth.normal_t(self.tag("q"), (1, Q, H, D), dtype=bf, device=dev)
+        self.qI = synth.normal_t(self.tag("qI"), (1, Q, HI, DI), dtype=bf, device=dev)
+        self.w = synth.normal_t(self.tag("w"), (1, Q, HI), std=1.0 / 8, device=dev)
+        self.idx = torch.empty((1, Q, self.K), dtype=torch.int32, device=dev)
+        self.out = torch.empty((1, Q, H, DV), dtype=bf, device=dev)
+        self.ws_i = L.workspace(L.lcs_workspace_size(L.OP_INDEX_TOPK, 1, Q, self.NC, 0, self.K), dev)
+        self.ws_a = L.workspace(L.lcs_workspace_size(L.OP_ATTEND, 1, Q, self.NC, TW, self.K, H, DV), dev)
+        torch.cuda.synchronize()
+
+    def _compress(self, stream):
+        L = self.lcs
+        n0 = self.P0 // 4
+        L.csa_compress(self.x, self.z, self.bias, m=4, overlap=2, d_rope=64, pos0=self.P0, x_tail=self.x_tail,
+                       z_tail=self.z_tail, out=self.comp[:, n0:], stream=stream)
+        L.csa_compress(self.kx, self.zI, self.biasI, m=4, overlap=2, d_rope=0, pos0=self.P0, x_tail=self.kx_tail,
+                       z_tail=self.zI_tail, out=self.kI[:, n0:], stream=stream)
+
+    def _index(self, stream):
+        L = self.lcs
+        L._call("csa_index_topk", L._ptr(self.qI), L.BF16, L._ptr(self.w), L._ptr(self.kI), L.BF16, 1, self.Q,
+                self.NC, HI, DI, L._ptr(self.q_pos), 4, self.K, L.F32, L._ptr(self.idx), None, L._ptr(self.ws_i),
+                self.ws_i.numel(), L._stream(stream))
+
+    def _attend(self, stream):
+        L = self.lcs
+        L._call("csa_attend", L._ptr(self.q), L.BF16, L._ptr(self.comp), L._ptr(self.win), L.BF16, 1, self.Q,
+                self.NC, self.win.shape[1], L._ptr(self.idx), self.K, L._ptr(self.q_pos), L._ptr(self.win_pos0),
+                TW, H, D, DV, SCALE, L._ptr(self.out), L.BF16, None, L._ptr(self.ws_a), self.ws_a.numel(),
+                L._stream(stream))
+
+    def step(self, stream):
+        self._compress(stream)
+        self._index(stream)
+        self._attend(stream)
+
+    def stage(self, name, stream):
+        {"compress": self._compress, "index": self._index, "topk": self._index, "attend": self._attend}[name](stream)
+
+    def units_per_step(self):
+        return self.Q
+
+    def pairs(self):
+        return sum(min(self.NC, (self.P0 + i + 1) // 4) for i in range(self.Q))
+
+    def alg_flops_per_step(self):
+        idx = self.pairs() * HI * DI * 2
+        att = self.Q * (self.K + TW) * H * (D + DV) * 2
+        return idx + att
+
+    def dominant_flops(self):
+        return self.pairs() * HI * DI * 2
+
+    def e2e_io(self):
+        return [self.x, self.kx, self.z, self.zI, self.q, self.qI, self.w], self.out
+
+    def cpu_sample(self, budget_s):
+        """Whole queries (index over their available entries, top-k, attention), first
+        and last queries of the chunk alternately, until the budget; compression excluded."""
+        from oracle import oracle as orc
+        comp = self.comp[0].double().cpu().numpy()
+        kI = self.kI[0].double().cpu().numpy()
+        win = self.win[0].double().cpu().numpy()
+        el, n = 0.0, 0
+        order = [i // 2 if i % 2 == 0 else self.Q - 1 - i // 2 for i in range(self.Q)]
+        for t in order:
+            if el >= budget_s:
+                break
+            pos = self.P0 + t
+            na = min(self.NC, (pos + 1) // 4)
+            qI = self.qI[0, t].double().cpu().numpy()
+            w = self.w[0, t].cpu().numpy()
+            q = self.q[0, t].double().cpu().numpy()
+            ts = time.perf_counter()
+            s = orc.index_scores_bf16(qI, w, kI[:na])
+            idx = orc.topk(s, self.K)
+            orc.csa_attend(q, comp, idx, win, self.P0 - 127, pos, TW, DV, SCALE)
+            el += time.perf_counter() - ts
+            n += 1
+        return n, el, f"{n} of {self.Q} queries (first and last of the chunk), index over their available " \
+                      f"entries, top-{self.K}, attention; compression excluded; single thread"
+
+
+class CompressStream(Workload):
+    """1M raw rows: CSA and HCA compression of the KV, CSA compression of the index keys."""
+    name = "compress_stream_1m"
+    unit = "tok/s"
+    T = 1 << 20
+    stage_names = ("csa_kv", "csa_index_keys", "hca_kv")
+    dominant = "compress_kernel"
+
+    def config(self):
+        return dict(workload=self.name, raw_tokens=self.T, kv_dim=D, index_dim=DI, csa_m=4, csa_overlap=2,
+                    hca_m=128, d_rope=64, kv_format="bf16")
+
+    def build(self):
+        import torch
+        from long_context_sparse_06_b200 import synth
+        dev, bf = self.dev, torch.bfloat16
+        T = self.T
+        self.x = synth.normal_t(self.tag("x"), (1, T, D), dtype=bf, device=dev)
+        self.kx = synth.normal_t(self.tag("kx"), (1, T, DI), dtype=bf, device=dev)
+        self.z = synth.normal_t(self.tag("z"), (1, T), device=dev)
+        self.zI = synth.normal_t(self.tag("zI"), (1, T), device=dev)
+        self.zh = synth.normal_t(self.tag("zh"), (1, T), device=dev)
+        self.bias = synth.normal_t(self.tag("bias"), (6,), device=dev)
+        self.biasI = synth.normal_t(self.tag("biasI"), (6,), device=dev)
+        self.biash = synth.normal_t(self.tag("biash"), (128,), device=dev)
+        self.csa = torch.empty((1, T // 4, D), dtype=bf, device=dev)
+        self.csaI = torch.empty((1, T // 4, DI), dtype=bf, device=dev)
+        self.hca = torch.empty((1, T // 128, D), dtype=bf, device=dev)
+
+    def _csa_kv(self, stream):
+        self.lcs.csa_compress(self.x, self.z, self.bias, m=4, overlap=2, d_rope=64, out=self.csa, stream=stream)
+
+    def _csa_keys(self, stream):
+        self.lcs.csa_compress(self.kx, self.zI, self.biasI, m=4, overlap=2, d_rope=0, out=self.csaI, stream=stream)
+
+    def _hca(self, stream):
+        self.lcs.hca_compress(self.x, self.zh, self.biash, m=128, d_rope=64, out=self.hca, stream=stream)
+
+    def step(self, stream):
+        self._csa_kv(stream)
+        self._csa_keys(stream)
+        self._hca(stream)
+
+    def stage(self, name, stream):
+        {"compress": self._csa_kv, "csa_kv": self._csa_kv, "csa_index_keys": self._csa_keys,
+         "hca_kv": self._hca}[name](stream)
+
+    def units_per_step(self):
+        return self.T
+
+    def alg_bytes_per_step(self):
+        T = self.T
+        return 2 * T * D * 2 + T * DI * 2 + 3 * T * 4 + (T // 4) * (D + DI) * 2 + (T // 128) * D * 2
+
+    def dominant_bytes(self):
+        T = self.T
+        return T * D * 2 + T * 4 + (T // 4) * D * 2
+
+    def e2e_io(self):
+        return [self.z, self.zI, self.zh], self.hca
+
+    def cpu_sample(self, budget_s):
+        from oracle import oracle as orc
+        el, n = 0.0, 0
+        rows = 4096
+        while el < budget_s and n + rows <= self.T:
+            x = self.x[0, n:n + rows].double().cpu().numpy()
+            z = self.z[0, n:n + rows].double().cpu().numpy()
+            b = self.bias.double().cpu().numpy()
+            ts = time.perf_counter()
+            orc.compress(x, z, b, 4, 2, d_rope=64, pos0=n)
+            el += time.perf_counter() - ts
+            n += rows
+        # the sample covers the CSA KV compression only; its rows/s is scaled by that
+        # pass's share of the step's algorithmic bytes
+        share = (self.T * D * 2) / self.alg_bytes_per_step()
+        return n * share, el, f"CSA compression of {n} raw rows of the KV (one of the three passes), rows/s " \
+                              f"scaled by that pass's share of the step's bytes; single thread"
+
+
+WORKLOADS = {c.name: c for c in (CsaDecode, HcaDecode, CsaDecodeMixed, CsaPrefill, CompressStream)}
+LAUNCHES_PER_STEP = {"csa_decode_bf16_128k": 4, "csa_decode_mixed_1m": 5, "hca_decode_bf16_1m": 2,
+                     "csa_prefill_bf16_8k": 5, "compress_stream_1m": 3}
+
+
+# ------------------------------------------------------------------- GPU arm
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -179,15 +570,23 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     lcs.lib()
-
-    x = make_inputs(dev, rank)
-    out = torch.empty((B, H, DV), dtype=torch.bfloat16, device=dev)
-    ws = lcs.workspace(lcs.lcs_workspace_size(lcs.OP_DECODE, B, 1, NC, TW, K, H, DV, lcs.F32), dev)
+    wl = WORKLOADS[args.workload](lcs, dev, rank)
+    wl.build()
     stream = torch.cuda.current_stream(dev)
 
-    def step(stream=None):
-        lcs.decode_fused(lcs.MODE_CSA, x["q"], x["comp"], x["win"], DV, SCALE, qI=x["qI"], w=x["w"], kI=x["kI"],
-                         k=K, out=out, ws=ws, stream=stream or torch.cuda.current_stream(dev))
+    if args.stage:
+        # one stage alone: warm-up, then K launches (for profilers; prints timing only)
+        for _ in range(args.warmup):
+            wl.stage(args.stage, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            wl.stage(args.stage, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        print(json.dumps({"workload": wl.name, "stage": args.stage, "ms": e0.elapsed_time(e1) / args.steps}))
+        return None
 
     def barrier():
         if world > 1:
@@ -200,24 +599,25 @@ def run_gpu(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
+    workspaces = [getattr(wl, a) for a in ("ws", "ws_i", "ws_a") if hasattr(wl, a)]
     for _ in range(args.warmup):
-        step()
+        wl.step(stream)
     torch.cuda.synchronize()
-    st = lcs.lcs_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status after warm-up: {st}")
+    for ws in workspaces:
+        st = lcs.lcs_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status after warm-up: {st}")
 
-    # One decode step (index -> top-k -> attention, chained with programmatic
-    # dependent launch) captured once as a CUDA graph and replayed: the decode
-    # loop is launch-bound on the host otherwise.
+    # The step captured once as a CUDA graph and replayed: decode loops are launch-bound
+    # on the host otherwise.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        step()
+        wl.step(torch.cuda.current_stream(dev))
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps of the whole path, inputs (297 MB/step) larger than L2
+    # ---- timed region: K steps of the whole path (inputs larger than L2)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     barrier()
@@ -229,50 +629,26 @@ def run_gpu(args):
         e1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
-    ms_step = ms_total / args.steps
-    value = world * B / (ms_step / 1e3)
+    ms_step = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    value = world * wl.units_per_step() / (ms_step / 1e3)
 
-    # ---- per-stage device time of the same step: events recorded by the library
-    # between its stages on the launching stream (direct calls; the stages then run
-    # without the programmatic overlap, so these sum to a little more than the step)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    for e in evs:   # torch creates the CUDA event on its first record
-        e.record(stream)
-    torch.cuda.synchronize()
-    handles = (lcs.C.c_void_p * 4)(*[e.cuda_event for e in evs])
-    stage_ms = [0.0, 0.0, 0.0]
-    lcs.lib().lcs_set_stage_events(handles, 4)
-    try:
-        for _ in range(3):
-            step()
-        torch.cuda.synchronize()
-        for _ in range(args.steps):
-            step()
-            torch.cuda.synchronize()
-            for i in range(3):
-                stage_ms[i] += evs[i].elapsed_time(evs[i + 1])
-    finally:
-        lcs.lib().lcs_set_stage_events(None, 0)
-    stage_ms = [max_over_ranks(s_ / args.steps) for s_ in stage_ms]
+    # ---- stage times on the launching stream (library events between stages, or events
+    # around separate calls); stages then run without programmatic overlap
+    stage_ms = time_stages(wl, lcs, stream, args.steps, torch)
+    stage_ms = {k: max_over_ranks(v) for k, v in stage_ms.items()}
 
     # ---- end to end through the public API: per-step inputs H2D from pinned host, result D2H
-    hq = x["q"].cpu().pin_memory()
-    hqI = x["qI"].cpu().pin_memory()
-    hw = x["w"].cpu().pin_memory()
-    hwin_row = x["win"][:, -1].contiguous().cpu().pin_memory()
-    hout = torch.empty((B, H, DV), dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hqI, hw, hwin_row))
+    ins, res_t = wl.e2e_io()
+    hosts = [t.cpu().pin_memory() for t in ins]
+    hout = torch.empty(res_t.shape, dtype=res_t.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hosts)
     d2h = hout.numel() * hout.element_size()
-    win_last = x["win"][:, -1]
 
     def e2e_step():
-        x["q"].copy_(hq, non_blocking=True)
-        x["qI"].copy_(hqI, non_blocking=True)
-        x["w"].copy_(hw, non_blocking=True)
-        win_last.copy_(hwin_row, non_blocking=True)
+        for d_, h_ in zip(ins, hosts):
+            d_.copy_(h_, non_blocking=True)
         graph.replay()
-        hout.copy_(out, non_blocking=True)
+        hout.copy_(res_t, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
         e2e_step()
@@ -285,37 +661,54 @@ def run_gpu(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-    st = lcs.lcs_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status after timing: {st}")
+    for ws in workspaces:
+        st = lcs.lcs_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status after timing: {st}")
     del graph
 
-    peak, peak_kind = load_peaks()
-    idx_bytes = B * index_bytes_per_request()
-    achieved = idx_bytes / (stage_ms[0] / 1e3) / 1e9
-    step_bytes = B * algorithmic_bytes_per_request()
+    hbm, tf_burst, tf_sust, peak_kind = load_peaks()
+    if wl.bound == "tensor":
+        dom_ms = stage_ms["index"]
+        achieved = wl.dominant_flops() / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": wl.dominant, "achieved": round(achieved, 1), "peak": tf_burst,
+                "unit": "TFLOP/s", "frac": round(achieved / tf_burst, 4), "peak_source": f"{peak_kind} bf16 burst",
+                "frac_of_sustained": round(achieved / tf_sust, 4),
+                "algorithmic_flops_per_launch": wl.dominant_flops(),
+                "traffic": recorded_traffic(wl.dominant, wl.name)}
+        step_flops = wl.alg_flops_per_step()
+        step_roof = {"algorithmic_flops_per_step": step_flops,
+                     "achieved_tflops": round(step_flops / (ms_step / 1e3) / 1e12, 1),
+                     "frac": round(step_flops / (ms_step / 1e3) / 1e12 / tf_burst, 4)}
+    else:
+        dom_ms = list(stage_ms.values())[wl.dominant_stage()]
+        achieved = wl.dominant_bytes() / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": wl.dominant, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": f"{peak_kind} copy bandwidth",
+                "algorithmic_bytes_per_launch": wl.dominant_bytes(),
+                "traffic": recorded_traffic(wl.dominant, wl.name)}
+        step_bytes = wl.alg_bytes_per_step()
+        step_roof = {"algorithmic_bytes_per_step": step_bytes,
+                     "achieved_gbs": round(step_bytes / (ms_step / 1e3) / 1e9, 1),
+                     "frac": round(step_bytes / (ms_step / 1e3) / 1e9 / hbm, 4)}
     res = None
     if rank == 0:
-        cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline(x)
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            n, el, sample = wl.cpu_sample(args.cpu_budget)
+            cpu = {"value": round(n / el, 4), "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": sample}
         res = {
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": round(value, 1), "unit": wl.unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))",
-            "config": dict(WORKLOAD, l2="inputs larger than L2 (297 MB/step vs 126 MB)",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 + Box-Muller)",
+            "config": dict(wl.config(), l2="inputs larger than L2 (126 MB) every step",
                            parallelism=f"replicas x{world} (requests independent)"),
-            "roofline": {"bound": "hbm", "kernel": "index_bf16_tc_kernel", "achieved": round(achieved, 1),
-                         "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "peak_source": peak_kind, "algorithmic_bytes_per_launch": idx_bytes,
-                         "traffic": recorded_traffic("index_bf16_tc_kernel")},
-            "step_roofline": {"algorithmic_bytes_per_step": step_bytes,
-                              "achieved_gbs": round(step_bytes / (ms_step / 1e3) / 1e9, 1),
-                              "frac": round(step_bytes / (ms_step / 1e3) / 1e9 / peak, 4)},
-            "stage_ms": {"index": round(stage_ms[0], 5), "topk": round(stage_ms[1], 5),
-                         "attend": round(stage_ms[2], 5)},
-            "e2e": {"value": round(world * B / (e2e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
-                    "inputs": "per-step q, qI, w and the new window row from pinned host; caches resident"},
-            "gpu_launches": args.steps * 4,
+            "roofline": roof, "step_roofline": step_roof,
+            "stage_ms": {k: round(v, 5) for k, v in stage_ms.items()},
+            "e2e": {"value": round(world * wl.units_per_step() / (e2e_ms / 1e3), 1), "unit": wl.unit,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
+                    "inputs": "per-step inputs H2D from pinned host, result D2H; caches resident"},
+            "gpu_launches": args.steps * LAUNCHES_PER_STEP[wl.name],
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,
         }
@@ -325,29 +718,70 @@ def run_gpu(args):
     return res
 
 
-def cpu_baseline(x, budget_s=20.0):
-    """The oracle, as it stands, on a bounded sample of the same workload: whole
-    requests, in order, until about budget_s seconds of oracle compute."""
-    from oracle import oracle as orc
-    el, n = 0.0, 0
-    while n < B and el < budget_s:
-        qI = x["qI"][n].double().cpu().numpy()
-        kI = x["kI"][n].double().cpu().numpy()
-        w = x["w"][n].cpu().numpy()
-        q = x["q"][n].double().cpu().numpy()
-        win = x["win"][n].double().cpu().numpy()
-        comp = x["comp"][n].double().cpu().numpy()
-        ts = time.perf_counter()
-        s = orc.index_scores_bf16(qI, w, kI)
-        idx = orc.topk(s, K)
-        orc.csa_attend(q, comp, idx, win, 0, -1, TW, DV, SCALE)
-        el += time.perf_counter() - ts
-        n += 1
-    return {"value": round(n / el, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} of {B} requests of the same workload, full path per request (index over all "
-                      f"{NC} entries, top-{K}, attention over {K}+{TW} rows); single thread"}
+def time_stages(wl, lcs, stream, steps, torch):
+    names = wl.stage_names
+    if isinstance(wl, (CsaDecode, HcaDecode)):
+        n_ev = len(names) + 1
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+        for e in evs:   # torch creates the CUDA event on its first record
+            e.record(stream)
+        torch.cuda.synchronize()
+        handles = (lcs.C.c_void_p * n_ev)(*[e.cuda_event for e in evs])
+        acc = [0.0] * len(names)
+        lcs.lib().lcs_set_stage_events(handles, n_ev)
+        try:
+            for _ in range(3):
+                wl.step(stream)
+            torch.cuda.synchronize()
+            for _ in range(steps):
+                wl.step(stream)
+                torch.cuda.synchronize()
+                for i in range(len(names)):
+                    acc[i] += evs[i].elapsed_time(evs[i + 1])
+        finally:
+            lcs.lib().lcs_set_stage_events(None, 0)
+        return {n: a / steps for n, a in zip(names, acc)}
+    if isinstance(wl, CsaPrefill):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for e in evs:
+            e.record(stream)
+        torch.cuda.synchronize()
+        handles = (lcs.C.c_void_p * 3)(*[e.cuda_event for e in evs])
+        acc = {n: 0.0 for n in names}
+        for _ in range(steps):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            wl._compress(stream)
+            a1.record(stream)
+            lcs.lib().lcs_set_stage_events(handles, 3)
+            try:
+                wl._index(stream)
+            finally:
+                lcs.lib().lcs_set_stage_events(None, 0)
+            b0.record(stream)
+            wl._attend(stream)
+            b1.record(stream)
+            torch.cuda.synchronize()
+            acc["compress"] += a0.elapsed_time(a1)
+            acc["index"] += evs[0].elapsed_time(evs[1])
+            acc["topk"] += evs[1].elapsed_time(evs[2])
+            acc["attend"] += b0.elapsed_time(b1)
+        return {n: v / steps for n, v in acc.items()}
+    fns = {"csa_kv": wl._csa_kv, "csa_index_keys": wl._csa_keys, "hca_kv": wl._hca}
+    acc = {n: 0.0 for n in names}
+    for _ in range(steps):
+        for n in names:
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            fns[n](stream)
+            a1.record(stream)
+            torch.cuda.synchronize()
+            acc[n] += a0.elapsed_time(a1)
+    return {n: v / steps for n, v in acc.items()}
 
 
+# ------------------------------------------------------------- reference arm
 def run_reference(args):
     """The oracle as the reference arm: each step is a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
@@ -357,8 +791,9 @@ def run_reference(args):
     import torch
     from long_context_sparse_06_b200 import synth
     from oracle import oracle as orc
-    # per-step sample: one request; the indexer over a contiguous slice of the entries,
-    # extrapolated to all NC entries; top-k and attention in full
+    if args.workload != "csa_decode_bf16_128k":
+        return {"impl": "reference", "unavailable": "the reference arm is timed on the headline workload only"}
+    NC, K = CsaDecode.NC, CsaDecode.K
     total_budget = 150.0
     per_step = total_budget / max(1, args.steps + args.warmup)
     probe = 2048
@@ -392,12 +827,14 @@ def run_reference(args):
     value = 1.0 / (ms / 1e3)
     sample = (f"1 request per step; indexer over {n_slice} of {NC} entries, time scaled to all entries; "
               f"top-{K} and attention over {K}+{TW} rows in full; single thread")
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 0,
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tok/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 where the oracle fixes it)",
-            "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))", "config": dict(WORKLOAD),
-            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(value, 4), "unit": UNIT},
-            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "data": "synthetic (seeded splitmix64 + Box-Muller, N(0,1))",
+            "config": {"workload": args.workload, "requests": 1, "compressed_entries": NC, "topk": K},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(value, 4),
+                             "unit": "tok/s"},
+            "e2e": {"value": round(value, 4), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def main():
@@ -406,9 +843,12 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lcs", choices=["lcs", "reference"])
+    ap.add_argument("--workload", default="csa_decode_bf16_128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--stage", default=None, help="run one stage alone (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
-    if args.warmup < 3:
+    if args.warmup < 3 and not args.stage:
         args.warmup = 3
     res = run_reference(args) if args.impl == "reference" else run_gpu(args)
     if res is not None:

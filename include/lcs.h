@@ -264,9 +264,12 @@ LCS_API int lcs_clear_status(void* ws, cudaStream_t stream);
 LCS_API const char* lcs_error_string(int code);
 
 /*
- * Profiling hook: when n >= 2 events are registered, decode_fused records
- * events[0] before its first stage, events[i] after stage i (i >= 1, up to
- * n-1), on the call's stream.  Pass n = 0 to stop.  Not thread-safe.
+ * Profiling hook: when n >= 2 events are registered, decode_fused and
+ * csa_index_topk record events[0] before their first stage and events[i] after
+ * stage i (i >= 1, up to n-1) on the call's stream (decode_fused CSA: index,
+ * top-k, attention; HCA: attention; csa_index_topk: index, top-k).  Stages are
+ * then launched without programmatic overlap.  Pass n = 0 to stop.  Not
+ * thread-safe.
  */
 LCS_API int lcs_set_stage_events(cudaEvent_t const* events, int n);
 

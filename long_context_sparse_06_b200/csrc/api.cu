@@ -283,10 +283,15 @@ int csa_index_topk(const void* qI, int qI_dtype, const float* w, const void* kI,
     if (!device_ok()) return LCS_ERR_CUDA;
     uint8_t* base = static_cast<uint8_t*>(ws);
     void* sc = scores ? scores : base + p.scores_off;
+    record_stage(0, stream);
     int r = run_index(qI, qI_dtype, w, kI, kI_dtype, B, Q, N_c, H_I, d_I, q_pos, m, sc, base + p.qscratch_off,
                       status_of(ws), stream, false);
     if (r != LCS_OK) return r;
-    return from_cuda(launch_topk(sc, score_dtype, B, Q, N_c, q_pos, m, k, idx, nullptr, status_of(ws), stream, true));
+    record_stage(1, stream);
+    r = from_cuda(launch_topk(sc, score_dtype, B, Q, N_c, q_pos, m, k, idx, nullptr, status_of(ws), stream,
+                              g_n_stage_events == 0));
+    record_stage(2, stream);
+    return r;
 }
 
 int lcs_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, int64_t N_c, const int64_t* q_pos, int m,

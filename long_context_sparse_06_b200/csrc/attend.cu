@@ -14,6 +14,7 @@
 //    tcgen05.mma with the query heads as M = 64:
 //      S [64 heads x 64 rows] = Q [64 x 576] . K_chunk^T        (K-major x K-major)
 //      O [64 heads x 512]    += P [64 x 64 rows] . V_chunk       (K-major x MN-major)
+//    with P = P_hi + P_lo, two bf16 parts, so P.V is two MMAs per chunk;
 //    O lives in TMEM as two interleaved M=64 accumulators (dims 0-255 in lanes
 //    0-15 of each 32-lane quarter, dims 256-511 in lanes 16-31), S beside it;
 //  * warps 4-7 gather the chunk's rows into a 2-stage ring with 16-byte
@@ -21,8 +22,9 @@
 //    bf16), writing the SW128 layout that both MMAs read (the same bytes are
 //    the K-major B of Q.K^T and the MN-major B of P.V);
 //  * warps 0-3 run the online softmax on S (fp32, exp2; S double-buffered in
-//    TMEM so Q.K^T of the next chunk overlaps it), write P as bf16 into the
-//    chunk's RoPE column block (dead once Q.K^T has read it), rescale O in TMEM
+//    TMEM so Q.K^T of the next chunk overlaps it), write P_hi into the
+//    chunk's RoPE column block (dead once Q.K^T has read it) and P_lo into a
+//    block of its own, rescale O in TMEM
 //    only when a head's running max grows by more than 2^8 in weight, and
 //    finally normalise O and write it out (or a split partial for the combine)
 //    through shared memory, so the global stores are coalesced.
@@ -41,7 +43,7 @@ constexpr int kBlk = kChunk * 128;            // one SW128 column block of a chu
 constexpr int kStageBytes = 9 * kBlk;         // 72 KB
 constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
 constexpr int kAtThreads = 320;   // 4 softmax, 4 gather, 1 Q.K^T issuer, 1 P.V issuer
-constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes;
+constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kBlk;   // + the low part of P
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
 
@@ -101,6 +103,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* q_s = smem;
     uint8_t* stage_s = smem + kQBytes;
+    uint8_t* plo_s = stage_s + 2 * kStageBytes;   // low bf16 part of P (one block)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g = blockIdx.x / splits;
@@ -219,14 +222,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 if (!mbar_wait(&bars.pfull[st], (uint32_t)((c >> 1) & 1), status, 303)) break;
                 tc_fence_after();
                 const uint64_t pd = k_desc0 + (uint64_t)((st * kStageBytes + 8 * kBlk) >> 4);
+                const uint64_t pld = k_desc0 + (uint64_t)((2 * kStageBytes) >> 4);
                 const uint64_t vd = v_desc0 + (uint64_t)((st * kStageBytes) >> 4);
 #pragma unroll
                 for (int half = 0; half < 2; ++half)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + (half ? (16u << 16) : 0u), pd + (uint64_t)((kk * 32) >> 4),
-                                    vd + (uint64_t)((half * 4 * kBlk + kk * 2048) >> 4), idesc_pv,
-                                    (c | kk) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t od = tmem + (half ? (16u << 16) : 0u);
+                        const uint64_t vk = vd + (uint64_t)((half * 4 * kBlk + kk * 2048) >> 4);
+                        mma_bf16_ss(od, pd + (uint64_t)((kk * 32) >> 4), vk, idesc_pv, (c | kk) ? 1u : 0u);
+                        mma_bf16_ss(od, pld + (uint64_t)((kk * 32) >> 4), vk, idesc_pv, 1u);
+                    }
                 mma_commit(&bars.kempty[st]);
                 mma_commit(&bars.ofull[st]);
             }
@@ -334,8 +340,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 rescale = (c > 0);
                 m_used = m_new;
             }
-            // P = bf16(exp2(scale*log2e*s - m)), written into the chunk's RoPE column block
-            // (dead once Q.K^T has read it): K-major SW128 rows of 128 B per head.
+            // p = exp2(scale*log2e*s - m) as two bf16 parts, p ~ hi + lo (relative error
+            // about 2^-17; a single bf16 P costs 2^-9 per weight, which heavy-tailed V turns
+            // into output errors near 2e-2 of the output RMS).  hi goes into the chunk's RoPE
+            // column block (dead once Q.K^T has read it), lo into the one P_lo block; both are
+            // K-major SW128 rows of 128 B per head.
             uint8_t* pblk = stage_s + st * kStageBytes + 8 * kBlk;
             float psum = 0.f;
 #pragma unroll
@@ -347,18 +356,35 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                     const float p0 = (cbase + j < nvalid) ? exp2f(__uint_as_float(sv[j]) * sl2 - m_used) : 0.f;
                     const float p1 = (cbase + j + 1 < nvalid) ? exp2f(__uint_as_float(sv[j + 1]) * sl2 - m_used) : 0.f;
                     pk[q] = pack_bf16x2(p0, p1);
-                    psum += bf16_bits_to_f32((uint16_t)(pk[q] & 0xFFFF)) + bf16_bits_to_f32((uint16_t)(pk[q] >> 16));
+                    const float h0 = bf16_bits_to_f32((uint16_t)(pk[q] & 0xFFFF));
+                    const float h1 = bf16_bits_to_f32((uint16_t)(pk[q] >> 16));
+                    sv[j] = __float_as_uint(p0 - h0);          // exact residuals
+                    sv[j + 1] = __float_as_uint(p1 - h1);
+                    psum += p0 + p1;
                 }
                 *reinterpret_cast<uint4*>(pblk + sw128_off(head, (cbase >> 3) + ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            // P_lo is single-buffered: the previous chunk's P.V must have read it.  (P.V of
+            // chunk c-3 is complete here -- chunk c-1 was gathered after it -- so the
+            // per-chunk-parity barrier cannot be two phases behind.)
+            if (c > 0) {
+                if (!mbar_wait(&bars.ofull[(c - 1) & 1], (uint32_t)(((c - 1) >> 1) & 1), status, 321)) break;
+                tc_fence_after();
+            }
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int j = ch * 8 + 2 * q;
+                    pk[q] = pack_bf16x2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                }
+                *reinterpret_cast<uint4*>(plo_s + sw128_off(head, (cbase >> 3) + ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             psum += __shfl_xor_sync(0xffffffffu, psum, 16);
             l_sum = l_sum * alpha + psum;
             if (__any_sync(0xffffffffu, rescale)) {
-                // O must be stable before it is rescaled: wait for the previous chunk's P.V.
-                // (P.V of chunk c-3 is complete here -- chunk c-1 was gathered after it -- so
-                // the per-chunk-parity barrier cannot be two phases behind.)
-                if (!mbar_wait(&bars.ofull[(c - 1) & 1], (uint32_t)(((c - 1) >> 1) & 1), status, 321)) break;
-                tc_fence_after();
+                // O is stable (the previous chunk's P.V is complete, waited for above).
                 const float f = rescale ? alpha : 1.f;
                 for (int j = 0; j < 256 / 16; ++j) {
                     uint32_t ov[16];

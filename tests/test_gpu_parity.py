@@ -404,3 +404,57 @@ def test_determinism_and_batch_invariance(L):
     L.decode_fused(L.MODE_CSA, q[1:2].contiguous(), comp[1:2].contiguous(), win[1:2].contiguous(), dv, scale,
                    qI=qI[1:2].contiguous(), w=w[1:2].contiguous(), kI=kI[1:2].contiguous(), k=k, idx_out=i4)
     assert torch.equal(i4[0], i1[1])
+
+
+# ------------------------------------------------------------- FP4 QK path
+def _fp4_keys(L, orc, name, B, Nc):
+    from long_context_sparse_06_b200 import synth
+    raw = synth.with_outliers(name, synth.normal(name, (B, Nc, 128))).astype(np.float32)
+    planes = L.lcs_quant_fp4(torch.from_numpy(raw).to(DEV))
+    p, s = orc.quant_fp4(raw.reshape(B * Nc, 128))
+    got = planes.cpu().numpy()
+    np.testing.assert_array_equal(got[:B * Nc * 64].reshape(B * Nc, 64), p)
+    np.testing.assert_array_equal(got[B * Nc * 64:].reshape(B * Nc, 4), s)
+    return planes, p.reshape(B, Nc, 64), s.reshape(B, Nc, 4)
+
+
+def test_index_fp4_bit_exact(L, orc):
+    """FP4 keys and on-the-fly FP4 query: bf16 scores and the selection bit-exact."""
+    B, H, Nc, k = 2, 64, 2000, 256
+    qI = randn("g.i4.q", (B, 1, H, 128), dtype=torch.bfloat16)
+    w = randn("g.i4.w", (B, 1, H), std=1 / 8)
+    planes, kp, ks = _fp4_keys(L, orc, "g.i4.k", B, Nc)
+    idx, sc = L.csa_index_topk(qI.to(DEV), w.to(DEV), planes, k, N_c=Nc, kI_dtype=L.FP4, want_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.float().cpu().numpy()
+    for b in range(B):
+        ref = orc.index_scores_fp4(qI[b, 0].float().numpy(), w[b, 0].numpy(), kp[b], ks[b])
+        np.testing.assert_array_equal(sc[b, 0], ref)
+        np.testing.assert_array_equal(idx[b, 0], orc.topk(ref.astype(np.float32), k))
+
+
+def test_decode_fused_mixed_precision(L, orc):
+    """The 1M-context config's formats at a small size: FP8 KV with bf16 RoPE dims,
+    FP4 index keys, bf16 scores, k = 1024."""
+    B, H, D, dv, Nc, k, Tw = 2, 64, 576, 512, 3000, 1024, 128
+    from long_context_sparse_06_b200 import synth
+    scale = 1 / math.sqrt(576)
+    q = randn("g.c5.q", (B, H, D), dtype=torch.bfloat16)
+    comp32 = synth.with_outliers("g.c5.c", synth.normal("g.c5.c", (B, Nc, D))).astype(np.float32)
+    win32 = synth.with_outliers("g.c5.w", synth.normal("g.c5.w", (B, Tw, D))).astype(np.float32)
+    comp_g = L.lcs_quant_kv_fp8(torch.from_numpy(comp32).to(DEV))
+    win_g = L.lcs_quant_kv_fp8(torch.from_numpy(win32).to(DEV))
+    qI = randn("g.c5.qi", (B, 64, 128), dtype=torch.bfloat16)
+    w = randn("g.c5.wi", (B, 64), std=1 / 8)
+    planes, kp, ks = _fp4_keys(L, orc, "g.c5.k", B, Nc)
+    idx_out = torch.empty((B, k), dtype=torch.int32, device=DEV)
+    out = both_outputs(lambda od: L.decode_fused(L.MODE_CSA, q.to(DEV), comp_g, win_g, dv, scale, kv_dtype=L.KV_FP8,
+                                                 qI=qI.to(DEV), w=w.to(DEV), kI=planes, kI_dtype=L.FP4, k=k,
+                                                 idx_out=idx_out, out_dtype=od)).cpu().numpy()
+    idx = idx_out.cpu().numpy()
+    comp_d = orc.dequant_kv_fp8(orc.quant_kv_fp8(comp32))
+    win_d = orc.dequant_kv_fp8(orc.quant_kv_fp8(win32))
+    for b in range(B):
+        ref_s = orc.index_scores_fp4(qI[b].float().numpy(), w[b].numpy(), kp[b], ks[b])
+        np.testing.assert_array_equal(idx[b], orc.topk(ref_s.astype(np.float32), k))
+        o, _ = orc.csa_attend(q[b].double().numpy(), comp_d[b], idx[b], win_d[b], 0, -1, 128, dv, scale)
+        assert_close_rel_rms(out[b], o, 2e-2, f"mixed-precision b {b}")
