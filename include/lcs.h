@@ -51,6 +51,7 @@ extern "C" {
 #define LCS_ERR_TIMEOUT     -4   /* a device-side bounded wait ran out */
 #define LCS_ERR_DEVICE      -5   /* device-side check failed (index out of range) */
 #define LCS_ERR_WORKSPACE   -6   /* workspace missing or too small */
+#define LCS_ERR_TOO_LARGE   -7   /* needs more scratch than csa_attend_noalloc holds */
 
 /* ---- storage types ---- */
 #define LCS_F32   0   /* float32 */
@@ -189,6 +190,38 @@ LCS_API int hca_attend(const void* q, int q_dtype, const void* comp, const void*
                const int64_t* q_pos, const int64_t* win_pos0, int m, int W, int H, int D, int d_v,
                float scale, void* out, int out_dtype, float* lse,
                void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * csa_attend without a workspace argument.  The pages describe no such call:
+ * it exists for callers that cannot hand the library any device memory --
+ * e.g. a serving engine that reserved nearly all of HBM for its KV-cache pool
+ * at start-up (a later allocation would fail or fragment the pool), or a host
+ * program that links only this library and keeps no device allocator.
+ *
+ * Arguments, layouts, results and host-side validation are those of
+ * csa_attend, with (ws, ws_bytes) replaced by
+ *   status_out  optional device int (NULL = not wanted) that receives, in
+ *               stream order, this call's device status (0 or a LCS_ERR_*
+ *               code, as lcs_status would report it).
+ * Scratch: a fixed library-owned device array of LCS_NOALLOC_SCRATCH_BYTES per
+ * device (256-byte aligned) holding the status word and the split partials.
+ * A problem whose scratch exceeds it returns LCS_ERR_TOO_LARGE before anything
+ * is enqueued; on a 148-SM B200 every shape csa_attend accepts fits.
+ * The call itself makes no cudaMalloc / cudaFree and no allocating library
+ * call; it clears the status word (cudaMemsetAsync) before its kernels run.
+ * The first call on each device looks the array up with cudaGetSymbolAddress
+ * (with that device current), which may make the CUDA runtime load the
+ * module that holds the array; make that first call before any stream
+ * capture starts.  Returns LCS_ERR_CUDA if the lookup fails.
+ * All calls on one device share the array: calls that overlap in time (other
+ * streams, other host threads) race on it and must be serialised by the caller.
+ */
+#define LCS_NOALLOC_SCRATCH_BYTES (20u << 20)
+LCS_API int csa_attend_noalloc(const void* q, int q_dtype, const void* comp, const void* win, int kv_dtype,
+               int64_t B, int64_t Q, int64_t N_c, int64_t Tw, const int32_t* idx, int k,
+               const int64_t* q_pos, const int64_t* win_pos0, int W, int H, int D, int d_v,
+               float scale, void* out, int out_dtype, float* lse,
+               int* status_out, cudaStream_t stream);
 
 /*
  * Fused decode step: one new token per request, one call.

@@ -49,6 +49,7 @@ def lib():
             "csa_index_topk": [P, I, P, P, I, I64, I64, I64, I, I, P, I, I, I, P, P, P, SZ, P],
             "lcs_topk": [P, I, I64, I64, I64, P, I, I, P, P, SZ, P],
             "csa_attend": [P, I, P, P, I, I64, I64, I64, I64, P, I, P, P, I, I, I, I, F, P, I, P, P, SZ, P],
+            "csa_attend_noalloc": [P, I, P, P, I, I64, I64, I64, I64, P, I, P, P, I, I, I, I, F, P, I, P, P, P],
             "hca_attend": [P, I, P, P, I, I64, I64, I64, I64, P, P, I, I, I, I, I, F, P, I, P, P, SZ, P],
             "decode_fused": [I, I64, P, I, P, P, I, I64, I64, I, I, I, F, P, I, P, P, I, I, I, I, I, P, I, P, P, P,
                              SZ, P],
@@ -216,6 +217,25 @@ def csa_attend(q, comp, win, idx, d_v, scale, kv_dtype=None, q_pos=None, win_pos
         ws = workspace(lcs_workspace_size(OP_ATTEND, B, Q, N_c, Tw, k, H, d_v), q.device)
     _call("csa_attend", _ptr(q), _dt(q), _ptr(comp), _ptr(win), kv_dtype, B, Q, N_c, Tw, _ptr(idx), k, _ptr(q_pos),
           _ptr(win_pos0), W, H, D, d_v, scale, _ptr(out), _dt(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    return (out, lse) if want_lse else out
+
+
+def csa_attend_noalloc(q, comp, win, idx, d_v, scale, kv_dtype=None, q_pos=None, win_pos0=None, W=128,
+                       want_lse=False, out=None, out_dtype=None, status_out=None, stream=None):
+    """csa_attend on the library's fixed per-device scratch: for callers that cannot give
+    the library device memory (an engine whose HBM is all reserved for its KV-cache pool,
+    a host program with no device allocator).  Pass `out` (and `status_out`, an int32
+    device tensor of one element) to keep this wrapper allocation-free as well.  Calls
+    that overlap in time on one device race on the shared scratch."""
+    torch = _torch()
+    B, Q, H, D, kv_dtype, N_c, Tw = _attend_common(q, comp, win, kv_dtype, d_v)
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty((B, Q, H, d_v), dtype=out_dtype or q.dtype, device=q.device)
+    lse = torch.empty((B, Q, H), dtype=torch.float32, device=q.device) if want_lse else None
+    _call("csa_attend_noalloc", _ptr(q), _dt(q), _ptr(comp), _ptr(win), kv_dtype, B, Q, N_c, Tw, _ptr(idx), k,
+          _ptr(q_pos), _ptr(win_pos0), W, H, D, d_v, scale, _ptr(out), _dt(out), _ptr(lse), _ptr(status_out),
+          _stream(stream))
     return (out, lse) if want_lse else out
 
 

@@ -174,6 +174,7 @@ const char* lcs_error_string(int code) {
         case LCS_ERR_TIMEOUT: return "device-side wait timed out";
         case LCS_ERR_DEVICE: return "device-side check failed";
         case LCS_ERR_WORKSPACE: return "workspace missing or too small";
+        case LCS_ERR_TOO_LARGE: return "problem needs more scratch than the allocation-free entry point holds";
         default: return "unknown status";
     }
 }
@@ -357,6 +358,33 @@ int hca_attend(const void* q, int q_dtype, const void* comp, const void* win, in
     AttendArgs a{q, comp, win, kv_dtype, B, Q, N_c, Tw, nullptr, 0, q_pos, win_pos0, m, W, H, D, d_v, scale, out, lse,
                  out_dtype};
     return run_attend(a, q_dtype, out_dtype, ws, ws_bytes, kStatusBytes, stream, false);
+}
+
+// Allocation-free csa_attend: the same validation and kernels, with the scratch in
+// the library's fixed per-device array (noalloc.cu) instead of a caller workspace.
+int csa_attend_noalloc(const void* q, int q_dtype, const void* comp, const void* win, int kv_dtype, int64_t B,
+                       int64_t Q, int64_t N_c, int64_t Tw, const int32_t* idx, int k, const int64_t* q_pos,
+                       const int64_t* win_pos0, int W, int H, int D, int d_v, float scale, void* out, int out_dtype,
+                       float* lse, int* status_out, cudaStream_t stream) {
+    if (idx == nullptr || k < 0) return LCS_ERR_INVALID;
+    AttendArgs a{q, comp, win, kv_dtype, B, Q, N_c, Tw, idx, k, q_pos, win_pos0, 1, W, H, D, d_v, scale, out, lse,
+                 out_dtype};
+    int v = validate_attend(a, q_dtype, out_dtype);
+    if (v != LCS_OK) return v;
+    if (kStatusBytes + align256(attend_scratch_bytes(a)) > (int64_t)LCS_NOALLOC_SCRATCH_BYTES)
+        return LCS_ERR_TOO_LARGE;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    void* ws = nullptr;
+    v = noalloc_scratch(&ws);
+    if (v != LCS_OK) return v;
+    // The status word must start at zero; the partials are written before they are read.
+    if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return LCS_ERR_CUDA;
+    if (launch_attend(a, static_cast<uint8_t*>(ws) + kStatusBytes, status_of(ws), stream, false) != cudaSuccess)
+        return LCS_ERR_CUDA;
+    if (status_out != nullptr &&
+        cudaMemcpyAsync(status_out, ws, sizeof(int), cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return LCS_ERR_CUDA;
+    return LCS_OK;
 }
 
 // ------------------------------------------------------------- fused decode

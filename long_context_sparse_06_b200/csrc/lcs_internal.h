@@ -69,6 +69,10 @@ struct AttendArgs {
 int64_t attend_scratch_bytes(const AttendArgs& a);
 cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaStream_t s, bool pdl);
 
+// noalloc.cu -- device address of the fixed scratch array behind csa_attend_noalloc
+// for the current device (looked up once per device).  LCS_OK or LCS_ERR_CUDA.
+int noalloc_scratch(void** ptr);
+
 // Raises a kernel's dynamic shared-memory limit once per process and kernel (the
 // attribute call costs host time on every launch otherwise).
 cudaError_t set_smem_once(const void* kern, size_t bytes);

@@ -15,7 +15,7 @@ def rms(x):
 
 
 def assert_close_rel_rms(got, ref, rel=2e-2, what=""):
-    """bf16 / FP8 outputs: max-abs error within rel * RMS(ref) (the benchmark spec's tolerance)."""
+    """bf16 / FP8 outputs: max-abs error within rel * RMS(ref) (the stated bf16 / FP8 tolerance)."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
