@@ -8,26 +8,33 @@
 // one softmax over the union of the selected (or all available) compressed
 // rows and the window rows.
 //
-// Tensor-core path (H = 64, D = 576, d_v = 512; bf16 rows or FP8 rows):
-//  * one CTA per (query, split of its row list), rows processed in chunks of 64;
-//  * warp 8 loads the 64 query heads once (TMA, 128-byte swizzle) and issues
+// Tensor-core path (H = 64, D = 576, d_v = 512; bf16 rows or FP8 rows), 448 threads:
+//  * one CTA per (query, split of its row list); the row list is the window rows
+//    (padded to whole chunks of 64) followed by the selected (CSA) or available (HCA)
+//    compressed rows; the splits of a query form one thread-block cluster;
+//  * warp 12 loads the 64 query heads once (TMA, 128-byte swizzle) and issues
 //    tcgen05.mma with the query heads as M = 64:
 //      S [64 heads x 64 rows] = Q [64 x 576] . K_chunk^T        (K-major x K-major)
+//    warp 13 issues
 //      O [64 heads x 512]    += P [64 x 64 rows] . V_chunk       (K-major x MN-major)
-//    with P = P_hi + P_lo, two bf16 parts, so P.V is two MMAs per chunk;
-//    O lives in TMEM as two interleaved M=64 accumulators (dims 0-255 in lanes
-//    0-15 of each 32-lane quarter, dims 256-511 in lanes 16-31), S beside it;
-//  * warps 4-7 gather the chunk's rows into a 2-stage ring with 16-byte
-//    cp.async (bf16) or load-convert-store (FP8 rows: E4M3 x block scale ->
-//    bf16), writing the SW128 layout that both MMAs read (the same bytes are
-//    the K-major B of Q.K^T and the MN-major B of P.V);
-//  * warps 0-3 run the online softmax on S (fp32, exp2; S double-buffered in
-//    TMEM so Q.K^T of the next chunk overlaps it), write P_hi into the
-//    chunk's RoPE column block (dead once Q.K^T has read it) and P_lo into a
-//    block of its own, rescale O in TMEM
-//    only when a head's running max grows by more than 2^8 in weight, and
-//    finally normalise O and write it out (or a split partial for the combine)
-//    through shared memory, so the global stores are coalesced.
+//    with P = P_hi + P_lo, two bf16 parts, so P.V is two MMAs per chunk.  O lives in
+//    TMEM as two interleaved M=64 accumulators (dims 0-255 in lanes 0-15 of each
+//    32-lane quarter, dims 256-511 in lanes 16-31), S double-buffered beside it;
+//  * warps 4-11 fill a 2-stage ring, four warps per stage, writing the SW128 layout that
+//    both MMAs read (the same bytes are the K-major B of Q.K^T and the MN-major B of
+//    P.V): contiguous bf16 chunks (window rows, HCA's compressed rows) with one TMA tile
+//    load per 128-byte column block; selected rows with 16-byte cp.async (row gathers
+//    scale with the number of issuing warps, not with TMA); FP8 rows with
+//    load-convert-store (E4M3 x power-of-two block scale -> bf16, exact).  Q and the
+//    window chunks are fetched before the kernel waits for the preceding kernel
+//    (programmatic dependent launch): they do not depend on it;
+//  * warps 0-3 run the online softmax on S (fp32, exp2), write P_hi into the chunk's
+//    RoPE column block (dead once Q.K^T has read it) and P_lo into a block of its
+//    own, rescale O in TMEM only when a head's running max grows by more than 2^8
+//    in weight, and write O / l out through shared memory (coalesced);
+//  * with several splits each CTA writes its unnormalised O and (m, l) to the
+//    workspace; after a cluster barrier CTA r merges heads r, r+splits, ... in split
+//    order.
 // F32 path (C1-sized problems): CUDA cores, fp32 online softmax.
 #include <utility>
 
@@ -42,8 +49,15 @@ constexpr int kH = 64, kD = 576, kDv = 512, kChunk = 64;
 constexpr int kBlk = kChunk * 128;            // one SW128 column block of a chunk: 64 rows x 128 B
 constexpr int kStageBytes = 9 * kBlk;         // 72 KB
 constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
-constexpr int kAtThreads = 320;   // 4 softmax, 4 gather, 1 Q.K^T issuer, 1 P.V issuer
+constexpr int kAtThreads = 448;   // 4 softmax, 8 producers, 1 Q.K^T issuer, 1 P.V issuer
+constexpr int kWarpQK = 12, kWarpPV = 13;
 constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kBlk;   // + the low part of P
+constexpr int kMaxSplits = 16;                // splits of one query form one cluster
+constexpr int kOPitchF32 = kDv * 4 + 16;      // staged O rows (padded)
+constexpr int kOPitchBF16 = kDv * 2 + 16;
+static_assert(kH * kOPitchF32 <= 2 * kStageBytes, "staged O fits in the stages");
+static_assert((32 * kMaxSplits + 32) * 4 + 32 * kMaxSplits * 8 <= kBlk, "combine tables fit in the P_lo block");
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
 
@@ -94,27 +108,60 @@ __device__ __forceinline__ const uint8_t* row_ptr(const AttendArgs& a, int64_t b
     return static_cast<const uint8_t*>(a.win) + (b * a.Tw + p.win_lo + (r - p.nsel)) * row_bytes;
 }
 
+// Window rows of query g: the rows r of win[b] with win_pos0[b] + r in [t-W+1, t]
+// (decode, q_pos == NULL: every row).  They come first in the tensor-core path's row list.
+struct WinPlan {
+    int64_t win_lo, nwin;
+};
+__device__ __forceinline__ WinPlan plan_window(const AttendArgs& a, int64_t g) {
+    WinPlan p;
+    if (a.q_pos == nullptr) {
+        p.win_lo = 0;
+        p.nwin = a.Tw;
+    } else {
+        const int64_t b = g / a.Q;
+        const int64_t t = a.q_pos[g];
+        const int64_t wp0 = a.win_pos0[b];
+        int64_t lo = t - a.W + 1 - wp0, hi = t - wp0;
+        if (lo < 0) lo = 0;
+        if (hi > a.Tw - 1) hi = a.Tw - 1;
+        p.win_lo = lo;
+        p.nwin = hi >= lo ? hi - lo + 1 : 0;
+    }
+    return p;
+}
+// HCA: compressed entries available to query g.
+__device__ __forceinline__ int64_t hca_avail(const AttendArgs& a, int64_t g) {
+    if (a.q_pos == nullptr) return a.N_c;
+    const int64_t av = (a.q_pos[g] + 1) / a.m;
+    return av < 0 ? 0 : (av < a.N_c ? av : a.N_c);
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(kAtThreads, 1)
-    attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const AttendArgs a, int splits,
+    attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_c,
+                     const __grid_constant__ CUtensorMap map_w, const AttendArgs a, int splits,
                      float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ AtBars bars;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* q_s = smem;
     uint8_t* stage_s = smem + kQBytes;
-    uint8_t* plo_s = stage_s + 2 * kStageBytes;   // low bf16 part of P (one block)
+    uint8_t* plo_s = stage_s + 2 * kStageBytes;   // low bf16 part of P (one block); after the
+                                                  // main loop, the combine's small tables
+    float* fac_s = reinterpret_cast<float*>(plo_s);             // [32][kMaxSplits]
+    float* inv_s = fac_s + 32 * kMaxSplits;                     // [32]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g = blockIdx.x / splits;
-    const int sp = blockIdx.x - (int)(g * splits);
+    const int sp = blockIdx.x - (int)(g * splits);   // == rank in the query's cluster
     const int64_t b = g / a.Q;
     constexpr int row_bytes = FP8 ? 656 : kD * 2;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars.qfull, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars.kfull[i], 128);
+            mbar_init(&bars.kfull[i], 128);   // the stage's four producer warps
             mbar_init(&bars.kempty[i], 1);
             mbar_init(&bars.pfull[i], 128);
             mbar_init(&bars.sfull[i], 1);
@@ -124,10 +171,144 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         mbar_init(&bars.odone, 1);
         fence_barrier_init();
         prefetch_tmap(&map_q);
+        if constexpr (!FP8) {
+            prefetch_tmap(&map_c);
+            prefetch_tmap(&map_w);
+        }
     }
-    if (warp == 8) {
+    if (warp == kWarpQK) {
         tmem_alloc(&bars.tmem_base, 512);
         tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+
+    // ---- what does not depend on the preceding kernel: the window rows, which fill the
+    // first chunks of the row list (the last one padded), the chunk range of this split
+    // (planned for the longest selection), Q.
+    const WinPlan wp = plan_window(a, g);
+    const int64_t nwc = (wp.nwin + kChunk - 1) / kChunk;
+    const int64_t comp_max = (a.idx != nullptr) ? a.k : hca_avail(a, g);
+    const int64_t nch_max = nwc + (comp_max + kChunk - 1) / kChunk;
+    const int64_t cps = (nch_max + splits - 1) / splits;
+    const int64_t c_begin = sp * cps;
+    const bool q_wanted = c_begin < nch_max;
+    if (warp == kWarpQK && lane == 0 && q_wanted) {
+        mbar_arrive_expect_tx(&bars.qfull, kQBytes);
+        for (int blk = 0; blk < 9; ++blk)
+            tma_load_2d(q_s + blk * (kH * 128), &map_q, &bars.qfull, blk * 64, (int)(g * kH));
+    }
+    const int32_t* sel = (a.idx != nullptr) ? a.idx + g * a.k : nullptr;
+    int nsel = 0;   // valid after the selection scan
+    // Global chunk gc: window chunk (gc < nwc) or compressed chunk; rows beyond the valid
+    // count are padding (masked in the softmax).
+    auto chunk_valid = [&](int64_t gc) -> int {
+        const int64_t v = gc < nwc ? wp.nwin - gc * kChunk : (int64_t)nsel - (gc - nwc) * kChunk;
+        return (int)(v < kChunk ? v : kChunk);
+    };
+
+    // ---- producers: warps 4-7 fill stage 0 (local chunks 0, 2, ...), warps 8-11 stage 1.
+    // Contiguous bf16 chunks (window rows; HCA's compressed rows) are one TMA tile load per
+    // 128-byte column block, issued by the group's first thread; selected rows (CSA) are
+    // gathered with 16-byte cp.async, warp pw of the group owning rows pw, pw+4, ..., pw+60
+    // (lane i < 16 resolves row pw+4i); FP8 rows are loaded, converted to bf16 (exact with
+    // the power-of-two block scale) and stored.  All write the SW128 layout both MMAs read.
+    const bool producer = warp >= 4 && warp < 12;
+    const int pst = (warp - 4) >> 2, pw = (warp - 4) & 3;
+    auto contiguous = [&](int64_t gc) { return !FP8 && (gc < nwc || sel == nullptr); };
+    auto row_src = [&](int64_t gc, int rr) -> const uint8_t* {
+        if (rr >= chunk_valid(gc)) return nullptr;
+        if (gc < nwc)
+            return static_cast<const uint8_t*>(a.win) + (b * a.Tw + wp.win_lo + gc * kChunk + rr) * row_bytes;
+        const int64_t j = (gc - nwc) * kChunk + rr;
+        const int64_t e = sel ? (int64_t)__ldg(sel + j) : j;
+        return static_cast<const uint8_t*>(a.comp) + (b * a.N_c + e) * row_bytes;
+    };
+    auto my_row_src = [&](int64_t gc) -> const uint8_t* {
+        return (lane < 16 && !contiguous(gc)) ? row_src(gc, pw + 4 * lane) : nullptr;
+    };
+    // Fills stage pst with global chunk gc and arrives on kfull (the TMA bytes complete it).
+    auto fill = [&](int64_t gc, const uint8_t* my_src) {
+        uint8_t* dst = stage_s + pst * kStageBytes;
+        if (contiguous(gc)) {
+            if (pw == 0 && lane == 0) {
+                mbar_arrive_expect_tx(&bars.kfull[pst], kStageBytes);
+                const bool w = gc < nwc;
+                const int row0 = w ? (int)(b * a.Tw + wp.win_lo + gc * kChunk) : (int)(b * a.N_c + (gc - nwc) * kChunk);
+                for (int blk = 0; blk < 9; ++blk)
+                    tma_load_2d(dst + blk * kBlk, w ? &map_w : &map_c, &bars.kfull[pst], blk * 64, row0);
+            } else {
+                mbar_arrive(&bars.kfull[pst]);
+            }
+            return;
+        }
+        if constexpr (!FP8) {
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const int rr = pw + 4 * i;
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(
+                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), i));
+                const bool valid = src != nullptr;
+                const uint8_t* base = valid ? src : static_cast<const uint8_t*>(a.comp);
+                for (int ch = lane; ch < 72; ch += 32)
+                    cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), base + (valid ? ch * 16 : 0), valid);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+        } else {
+            // FP8 row: 32 content pieces of 16 codes (-> 32 bf16) and 8 RoPE pieces of 8 bf16;
+            // 8 rows' loads in flight per lane
+            for (int i0 = 0; i0 < 16; i0 += 8) {
+                uint4 cv[8], rv[8];
+                float sc[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint8_t* src = reinterpret_cast<const uint8_t*>(
+                        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), i0 + u));
+                    cv[u] = make_uint4(0, 0, 0, 0);
+                    rv[u] = make_uint4(0, 0, 0, 0);
+                    sc[u] = 0.f;
+                    if (src != nullptr) {
+                        cv[u] = __ldg(reinterpret_cast<const uint4*>(src + lane * 16));
+                        sc[u] = __ldg(reinterpret_cast<const float*>(src + 640) + (lane >> 3));
+                        if (lane < 8) rv[u] = __ldg(reinterpret_cast<const uint4*>(src + 512 + lane * 16));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int rr = pw + 4 * (i0 + u);
+                    const uint32_t w4[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        o[2 * q] =
+                            pack_bf16x2(e4m3_to_f32(w4[q] & 0xFF) * sc[u], e4m3_to_f32((w4[q] >> 8) & 0xFF) * sc[u]);
+                        o[2 * q + 1] =
+                            pack_bf16x2(e4m3_to_f32((w4[q] >> 16) & 0xFF) * sc[u], e4m3_to_f32(w4[q] >> 24) * sc[u]);
+                    }
+                    const int ch = lane * 2;
+                    *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(dst + ((ch + 1) >> 3) * kBlk + sw128_off(rr, (ch + 1) & 7)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
+                    if (lane < 8) *reinterpret_cast<uint4*>(dst + 8 * kBlk + sw128_off(rr, lane)) = rv[u];
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars.kfull[pst]);
+    };
+    // Window chunks need no selection: the first chunk of each stage is filled before the
+    // wait for the preceding kernel when it is a window chunk of this split.
+    bool pre = false;
+    if (producer) {
+        const int64_t gc = c_begin + pst;
+        if (pst < cps && gc < nch_max && gc < nwc) {
+            fill(gc, my_row_src(gc));
+            pre = true;
+        }
     }
 #if defined(__CUDA_ARCH__)
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -136,14 +317,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // An index >= N_c ends the prefix and is reported through the status word.
     if (a.idx != nullptr) {
         if (warp == 0) {
-            const int32_t* ir = a.idx + g * a.k;
             int first_bad = a.k;
             for (int base = 0; base < a.k; base += 256) {
                 int32_t v[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int i = base + 32 * j + lane;
-                    v[j] = (i < a.k) ? __ldg(ir + i) : 0;
+                    v[j] = (i < a.k) ? __ldg(sel + i) : 0;
                 }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -158,23 +338,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             if (lane == 0) bars.nsel = first_bad;
         }
     } else if (threadIdx.x == 0) {
-        int64_t n = a.N_c;
-        if (a.q_pos != nullptr) {
-            const int64_t av = (a.q_pos[g] + 1) / a.m;
-            n = av < 0 ? 0 : (av < a.N_c ? av : a.N_c);
-        }
-        bars.nsel = (int)n;
+        bars.nsel = (int)comp_max;
     }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = bars.tmem_base;
-    const int32_t* sel = (a.idx != nullptr) ? a.idx + g * a.k : nullptr;
-    const RowPlan plan = plan_rows(a, g, bars.nsel);
-    const int64_t R = plan.nsel + plan.nwin;
-    const int64_t nch_all = (R + kChunk - 1) / kChunk;
-    const int64_t cps = (nch_all + splits - 1) / splits;
-    const int64_t c_begin = sp * cps;
+    nsel = bars.nsel;
+    const int64_t nch_all = nwc + (nsel + kChunk - 1) / kChunk;
     const int64_t c_end = (c_begin + cps < nch_all) ? c_begin + cps : nch_all;
     const int nch = (int)(c_end > c_begin ? c_end - c_begin : 0);
 
@@ -184,20 +352,16 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // offset 16: two interleaved M=64 accumulators), S double-buffered in 256..383.
     auto t_s = [&](int buf) { return tmem + 256u + 64u * (uint32_t)buf; };
 
-    if (warp == 8) {
-        if (lane == 0 && nch > 0) {
-            // ---------------- Q load + MMA issue
-            mbar_arrive_expect_tx(&bars.qfull, kQBytes);
-            for (int blk = 0; blk < 9; ++blk)
-                tma_load_2d(q_s + blk * (kH * 128), &map_q, &bars.qfull, blk * 64, (int)(g * kH));
+    if (warp == kWarpQK) {
+        if (lane == 0 && q_wanted) {
+            // ---------------- Q.K^T issue
             bool ok = mbar_wait(&bars.qfull, 0, status, 300);
-            // descriptors: base once, then byte offsets >> 4 added to the start-address field
             const uint64_t q_desc = sw128_desc(smem_u32(q_s), 16, 1024);
             const uint64_t k_desc0 = sw128_desc(smem_u32(stage_s), 16, 1024);
-            auto issue_qk = [&](int c) -> bool {
+            for (int c = 0; c < nch && ok; ++c) {
                 const int st = c & 1;
-                if (!mbar_wait(&bars.kfull[st], (uint32_t)((c >> 1) & 1), status, 301)) return false;
-                if (c >= 2 && !mbar_wait(&bars.sempty[st], (uint32_t)(((c - 2) >> 1) & 1), status, 302)) return false;
+                if (!mbar_wait(&bars.kfull[st], (uint32_t)((c >> 1) & 1), status, 301)) break;
+                if (c >= 2 && !mbar_wait(&bars.sempty[st], (uint32_t)(((c - 2) >> 1) & 1), status, 302)) break;
                 tc_fence_after();
                 const uint64_t kd = k_desc0 + (uint64_t)((st * kStageBytes) >> 4);
 #pragma unroll
@@ -207,14 +371,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                         mma_bf16_ss(t_s(st), q_desc + (uint64_t)((blk * (kH * 128) + kk * 32) >> 4),
                                     kd + (uint64_t)((blk * kBlk + kk * 32) >> 4), idesc_qk, (blk | kk) ? 1u : 0u);
                 mma_commit(&bars.sfull[st]);
-                return true;
-            };
-            for (int c = 0; c < nch && ok; ++c) ok = issue_qk(c);
+            }
         }
-    } else if (warp == 9) {
+    } else if (warp == kWarpPV) {
         if (lane == 0 && nch > 0) {
             // ---------------- P.V issue (its own thread, so that it never waits behind the
-            // next chunk's Q.K^T, which waits for that chunk's gather)
+            // next chunk's Q.K^T, which waits for that chunk's gather); P = P_hi + P_lo
             const uint64_t k_desc0 = sw128_desc(smem_u32(stage_s), 16, 1024);
             const uint64_t v_desc0 = sw128_desc(smem_u32(stage_s), kBlk, 1024);
             for (int c = 0; c < nch; ++c) {
@@ -238,74 +400,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
             mma_commit(&bars.odone);
         }
-    } else if (warp >= 4) {
-        // ---------------- gather producer: warps 4..7.  Warp pw owns rows pw, pw+4, ..., pw+60 of
-        // a chunk; lane i first resolves the source of row pw+4i (one index load per row), then
-        // the warp streams each row with lanes on consecutive 16-byte pieces (coalesced).
-        const int pw = warp - 4;
-        for (int c = 0; c < nch; ++c) {
-            const int st = c & 1;
-            if (c >= 2 && !mbar_wait(&bars.kempty[st], (uint32_t)(((c - 2) >> 1) & 1), status, 310)) break;
-            uint8_t* dst = stage_s + st * kStageBytes;
-            const int64_t r0 = (c_begin + c) * kChunk;
-            const uint8_t* my_src = nullptr;
-            if (lane < 16) {
-                const int64_t r = r0 + pw + 4 * lane;
-                if (r < R) my_src = row_ptr(a, b, plan, sel, r, row_bytes);
-            }
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const int rr = pw + 4 * i;
-                const uint8_t* src = reinterpret_cast<const uint8_t*>(
-                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), i));
-                const bool valid = src != nullptr;
-                if constexpr (!FP8) {
-                    const uint8_t* base = valid ? src : static_cast<const uint8_t*>(a.comp);
-                    for (int ch = lane; ch < 72; ch += 32)
-                        cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), base + (valid ? ch * 16 : 0), valid);
-                } else {
-                    // FP8 row: 32 content pieces of 16 codes (-> 32 bf16, exact with the
-                    // power-of-two block scale) and 8 RoPE pieces of 8 bf16
-                    for (int seg = lane; seg < 40; seg += 32) {
-                        uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-                        if (valid) {
-                            if (seg < 32) {
-                                const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + seg * 16));
-                                const float sc = __ldg(reinterpret_cast<const float*>(src + 640) + (seg >> 3));
-                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                                uint32_t o[8];
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    o[2 * q] = pack_bf16x2(e4m3_to_f32(w4[q] & 0xFF) * sc,
-                                                           e4m3_to_f32((w4[q] >> 8) & 0xFF) * sc);
-                                    o[2 * q + 1] = pack_bf16x2(e4m3_to_f32((w4[q] >> 16) & 0xFF) * sc,
-                                                               e4m3_to_f32(w4[q] >> 24) * sc);
-                                }
-                                lo = make_uint4(o[0], o[1], o[2], o[3]);
-                                hi = make_uint4(o[4], o[5], o[6], o[7]);
-                            } else {
-                                lo = __ldg(reinterpret_cast<const uint4*>(src + 512 + (seg - 32) * 16));
-                            }
-                        }
-                        if (seg < 32) {
-                            const int ch = seg * 2;
-                            *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
-                            *reinterpret_cast<uint4*>(dst + ((ch + 1) >> 3) * kBlk + sw128_off(rr, (ch + 1) & 7)) = hi;
-                        } else {
-                            const int ch = 64 + (seg - 32);
-                            *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) = lo;
-                        }
-                    }
-                }
-            }
-            if constexpr (!FP8) {
-                cp_async_commit();
-                cp_async_wait<0>();
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&bars.kfull[st]);
+    } else if (producer) {
+        // ---------------- producer loop (the group's chunks pst, pst+2, ...); a stage is
+        // refilled once the P.V that read it is complete.  The next chunk's row sources are
+        // resolved while this chunk's copies are in flight.
+        const uint8_t* nxt = (pst < nch) ? my_row_src(c_begin + pst) : nullptr;
+        for (int c = pst; c < nch; c += 2) {
+            const uint8_t* my_src = nxt;
+            const int u = c >> 1;
+            if (u >= 1 && !mbar_wait(&bars.kempty[pst], (uint32_t)((u - 1) & 1), status, 310)) break;
+            if (c + 2 < nch) nxt = my_row_src(c_begin + c + 2);
+            if (!(pre && c == pst)) fill(c_begin + c, my_src);
         }
-    } else {
+    } else if (warp < 4) {
         // ---------------- softmax / correction / epilogue: warps 0..3.  Warp q owns heads
         // 16q..16q+15; lane l works on head 16q + (l & 15) and, with the 16x32bx2 TMEM
         // load, on S columns 0-31 (lanes 0-15) or 32-63 (lanes 16-31).
@@ -314,7 +421,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const int head = quarter * 16 + hl;
         const int cbase = (lane < 16) ? 0 : 32;   // this lane's S columns
         float m_used = -INFINITY;                 // log2-domain running max used for exponentials
-        float l_sum = 0.f;                        // sum of the bf16-rounded weights (both lane halves)
+        float l_sum = 0.f;                        // sum of the weights (both lane halves)
         const float sl2 = a.scale * kLog2e;
         for (int c = 0; c < nch; ++c) {
             const int st = c & 1;
@@ -325,8 +432,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&bars.sempty[st]);
-            const int64_t rbase = (c_begin + c) * kChunk;
-            const int nvalid = (int)((R - rbase) < kChunk ? (R - rbase) : kChunk);
+            const int nvalid = chunk_valid(c_begin + c);
             float mx = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -401,23 +507,22 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             fence_proxy_async_smem();
             mbar_arrive(&bars.pfull[st]);
         }
-        // ---- epilogue: O / l (or the split partial), staged through shared memory so that
-        // the global writes are coalesced.  Lane l of warp q holds O row of head 16q + (l & 15),
-        // dims 0-255 (lanes 0-15) or 256-511 (lanes 16-31).
-        const bool have = nch > 0;
-        if (have) mbar_wait(&bars.odone, 0, status, 322);
+        // ---- epilogue: O (normalised when this is the only split; else the partial O and
+        // (m, l) for the cluster combine) staged through shared memory, coalesced global
+        // writes.  Lane l of warp q holds the O row of head 16q + (l & 15), dims 0-255
+        // (lanes 0-15) or 256-511 (lanes 16-31).
+        if (nch > 0) mbar_wait(&bars.odone, 0, status, 322);
         tc_fence_after();
-        const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
-        const int dim0 = (lane < 16) ? 0 : 256;
         const bool final_out = splits == 1;
+        const float fs = final_out ? ((l_sum > 0.f) ? 1.f / l_sum : 0.f) : 1.f;
+        const int dim0 = (lane < 16) ? 0 : 256;
         const bool f32 = !final_out || a.out_dtype == LCS_F32;
-        const int row_pitch = f32 ? (kDv * 4 + 16) : (kDv * 2 + 16);   // padded rows: fewer bank conflicts
-        uint8_t* ostage = stage_s;                                     // stages are free after the last P.V
-        const float fs = final_out ? inv : 1.f;
+        const int row_pitch = f32 ? kOPitchF32 : kOPitchBF16;   // padded rows: fewer bank conflicts
+        uint8_t* ostage = stage_s;                               // stages are free after the last P.V
         uint8_t* rowp = ostage + head * row_pitch;
         for (int j0 = 0; j0 < 256 / 16; j0 += 4) {
             uint32_t ov[4][16];
-            if (have) {
+            if (nch > 0) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) tmem_ld16(tmem_addr(tmem, quarter * 32, (j0 + u) * 16), ov[u]);
                 tmem_ld_wait();
@@ -446,18 +551,18 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 }
             }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 epilogue warps
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 softmax warps
         const int row_bytes_out = f32 ? kDv * 4 : kDv * 2;
         uint8_t* gout = final_out ? static_cast<uint8_t*>(a.out) + g * kH * row_bytes_out
                                   : reinterpret_cast<uint8_t*>(part_o + (g * splits + sp) * kH * kDv);
-        const int t128 = threadIdx.x;   // 0..127
-        for (int off = t128 * 16; off < kH * row_bytes_out; off += 128 * 16) {
+        for (int off = (int)threadIdx.x * 16; off < kH * row_bytes_out; off += 128 * 16) {
             const int h = off / row_bytes_out, cb = off - h * row_bytes_out;
             *reinterpret_cast<uint4*>(gout + off) = *reinterpret_cast<const uint4*>(ostage + h * row_pitch + cb);
         }
         if (lane < 16) {
             if (final_out) {
-                if (a.lse != nullptr) a.lse[g * kH + head] = (l_sum > 0.f) ? (m_used + log2f(l_sum)) / kLog2e : -INFINITY;
+                if (a.lse != nullptr)
+                    a.lse[g * kH + head] = (l_sum > 0.f) ? (m_used + log2f(l_sum)) / kLog2e : -INFINITY;
             } else {
                 float* ml = part_ml + ((g * splits + sp) * kH + head) * 2;
                 ml[0] = (l_sum > 0.f) ? m_used : -INFINITY;
@@ -467,37 +572,90 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
-    if (warp == 8) {
+    if (splits > 1) {
+        // ---- cluster combine: the splits of query g are the CTAs of one cluster.  Once
+        // every split's partial is in global memory (L2), CTA r merges heads r, r+splits, ...
+        // in split order.
+        __threadfence();
+        cluster_sync_all();
+        const uint32_t rank = cluster_ctarank();
+        const int nh = (kH - (int)rank + splits - 1) / splits;
+        const float* mlq = part_ml + g * splits * kH * 2;
+        const float* oq = part_o + g * splits * kH * kDv;
+        // (m, l) of every (head of this CTA, split): one load each, all in flight together
+        float2* mls = reinterpret_cast<float2*>(inv_s + 32);   // [32][kMaxSplits]
+        for (int t = threadIdx.x; t < nh * splits; t += blockDim.x) {
+            const int j = t / splits, s = t - j * splits;
+            mls[j * kMaxSplits + s] = __ldcg(reinterpret_cast<const float2*>(mlq) + s * kH + (int)rank + splits * j);
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < nh; j += blockDim.x) {
+            const int h = (int)rank + splits * j;
+            float M = -INFINITY;
+            for (int s = 0; s < splits; ++s) M = fmaxf(M, mls[j * kMaxSplits + s].x);
+            float L = 0.f;
+            for (int s = 0; s < splits; ++s) {
+                const float2 ml = mls[j * kMaxSplits + s];
+                const float e = (ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
+                fac_s[j * kMaxSplits + s] = e;
+                L += ml.y * e;
+            }
+            inv_s[j] = L > 0.f ? 1.f / L : 0.f;
+            if (a.lse != nullptr) a.lse[g * kH + h] = L > 0.f ? (M + log2f(L)) / kLog2e : -INFINITY;
+        }
+        __syncthreads();
+        // O rows: a thread merges kItems (head, 4-dim) items at a time, their loads for one
+        // split in flight together
+        constexpr int kItems = 4;
+        const int n_items = nh * (kDv / 4);
+        for (int i0 = threadIdx.x; i0 < n_items; i0 += kItems * blockDim.x) {
+            float4 acc[kItems];
+#pragma unroll
+            for (int u = 0; u < kItems; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s < splits; ++s) {
+                float4 v[kItems];
+#pragma unroll
+                for (int u = 0; u < kItems; ++u) {
+                    const int item = i0 + u * blockDim.x;
+                    const int j = item / (kDv / 4), d4 = item - j * (kDv / 4);
+                    v[u] = item < n_items
+                               ? __ldcg(reinterpret_cast<const float4*>(oq + (s * kH + (int)rank + splits * j) * kDv) + d4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < kItems; ++u) {
+                    const int item = i0 + u * blockDim.x;
+                    const float e = item < n_items ? fac_s[(item / (kDv / 4)) * kMaxSplits + s] : 0.f;
+                    acc[u].x += v[u].x * e;
+                    acc[u].y += v[u].y * e;
+                    acc[u].z += v[u].z * e;
+                    acc[u].w += v[u].w * e;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kItems; ++u) {
+                const int item = i0 + u * blockDim.x;
+                if (item >= n_items) break;
+                const int j = item / (kDv / 4), d4 = item - j * (kDv / 4);
+                const int h = (int)rank + splits * j;
+                const float iv = inv_s[j];
+                const int64_t o = (g * kH + h) * kDv + d4 * 4;
+                if (a.out_dtype == LCS_F32) {
+                    *reinterpret_cast<float4*>(static_cast<float*>(a.out) + o) =
+                        make_float4(acc[u].x * iv, acc[u].y * iv, acc[u].z * iv, acc[u].w * iv);
+                } else {
+                    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + o) = make_uint2(
+                        pack_bf16x2(acc[u].x * iv, acc[u].y * iv), pack_bf16x2(acc[u].z * iv, acc[u].w * iv));
+                }
+            }
+        }
+    } else {
+        __syncthreads();
+    }
+    if (warp == kWarpQK) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-}
-
-// Merges the split partials of each (query, head) in split order (fixed tree:
-// sequential), writing bf16 output and the natural-log LSE.
-__global__ void attend_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                      int splits, void* __restrict__ out, int out_dtype, float* __restrict__ lse) {
-    const int64_t gh = blockIdx.x;   // (query, head)
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[(gh / kH * splits + s) * kH * 2 + (gh % kH) * 2]);
-    float L = 0.f;
-    for (int s = 0; s < splits; ++s) {
-        const float* ml = part_ml + (gh / kH * splits + s) * kH * 2 + (gh % kH) * 2;
-        if (ml[1] > 0.f) L += ml[1] * exp2f(ml[0] - M);
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int d = threadIdx.x; d < kDv; d += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < splits; ++s) {
-            const float* ml = part_ml + (gh / kH * splits + s) * kH * 2 + (gh % kH) * 2;
-            if (ml[1] > 0.f)
-                acc += part_o[((gh / kH * splits + s) * kH + gh % kH) * kDv + d] * exp2f(ml[0] - M);
-        }
-        if (out_dtype == LCS_F32) static_cast<float*>(out)[gh * kDv + d] = acc * inv;
-        else static_cast<uint16_t*>(out)[gh * kDv + d] = f32_to_bf16_bits(acc * inv);
-    }
-    if (lse != nullptr && threadIdx.x == 0) lse[gh] = L > 0.f ? (M + log2f(L)) / kLog2e : -INFINITY;
 }
 
 // --------------------------------------------------------------- fp32 path
@@ -590,20 +748,71 @@ __global__ void attend_f32_kernel(const AttendArgs a, int* status) {
             a.lse[g * H + h] = lh[h] > 0.f ? mh[h] + logf(lh[h]) : -INFINITY;
 }
 
+int64_t max_chunks(const AttendArgs& a) {
+    const int64_t nw = (a.q_pos == nullptr ? a.Tw : (a.W < a.Tw ? a.W : a.Tw));
+    return (nw + kChunk - 1) / kChunk + ((a.idx != nullptr ? a.k : a.N_c) + kChunk - 1) / kChunk;
+}
+
+const void* tc_kernel(const AttendArgs& a) {
+    return (a.kv_dtype == LCS_KV_FP8) ? reinterpret_cast<const void*>(attend_tc_kernel<true>)
+                                      : reinterpret_cast<const void*>(attend_tc_kernel<false>);
+}
+
+// How many clusters of `s` CTAs (one per SM: this kernel's shared memory) the device
+// keeps resident at once; cached per kernel and size.  Sizes above 8 are non-portable.
+int resident_clusters(const void* kern, int s) {
+    static std::mutex mu;
+    static int cache[2][kMaxSplits + 1];
+    const int which = (kern == reinterpret_cast<const void*>(attend_tc_kernel<true>));
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[which][s] == 0) {
+        int n = 0;
+        if (set_smem_once(kern, kAtSmem) == cudaSuccess &&
+            (s <= 8 || cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)s);
+            cfg.blockDim = dim3(kAtThreads);
+            cfg.dynamicSmemBytes = kAtSmem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)s;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+        }
+        cudaGetLastError();
+        cache[which][s] = n > 0 ? n : -1;
+    }
+    return cache[which][s];
+}
+
+// Splits per query: each query's splits form one cluster and every CTA of the launch is
+// resident at once (queries x splits <= SMs).  Picks the size that minimises the chunks
+// per CTA plus a fixed per-CTA cost of about two chunks (prologue, pipeline fill, epilogue
+// and combine), keeping at least two chunks per split.
 int choose_splits(const AttendArgs& a) {
     const int64_t queries = a.B * a.Q;
-    const int64_t rmax = (a.idx != nullptr ? a.k : a.N_c) + (a.q_pos == nullptr ? a.Tw : (a.W < a.Tw ? a.W : a.Tw));
-    const int64_t chunks = (rmax + kChunk - 1) / kChunk;
-    int64_t s = num_sms() / (queries > 0 ? queries : 1);
-    if (s < 1) s = 1;
-    if (s > chunks) s = chunks > 0 ? chunks : 1;
-    // at least two chunks per split so the ring overlaps gather and math
-    while (s > 1 && (chunks + s - 1) / s < 2) --s;
-    return (int)s;
+    const int64_t chunks = max_chunks(a);
+    const void* kern = tc_kernel(a);
+    int best = 1;
+    double best_cost = (double)chunks + 2.0;
+    for (int s = 2; s <= kMaxSplits; ++s) {
+        if ((chunks + s - 1) / s < 2 || queries * s > num_sms()) break;
+        if (resident_clusters(kern, s) < queries) continue;
+        const double cost = (double)((chunks + s - 1) / s) + 2.0;
+        if (cost < best_cost) {
+            best = s;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
 }  // namespace
 
+// Split partials: fp32 O [queries, splits, 64, 512] and (m, l) [queries, splits, 64, 2].
 int64_t attend_scratch_bytes(const AttendArgs& a) {
     if (a.kv_dtype == LCS_F32) return 0;
     const int s = choose_splits(a);
@@ -622,26 +831,58 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
         if (e != cudaSuccess) return e;
         return launch_k(attend_f32_kernel, dim3((unsigned)queries), dim3(256), smem, s, pdl, a, status);
     }
-    const int splits = choose_splits(a);
-    CUtensorMap mq;
+    CUtensorMap mq, mc, mw;
     if (!encode_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, kD, (uint64_t)(queries * kH), kD * 2, 64, kH,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    if (a.kv_dtype == LCS_BF16) {
+        // contiguous-row maps: boxes of 64 rows x 64 columns (128 B), 128-byte swizzle;
+        // row coordinates are int32
+        if (a.B * a.N_c >= (int64_t(1) << 31) || a.B * a.Tw >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+        if (!encode_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.comp, kD, (uint64_t)(a.B * a.N_c), kD * 2, 64,
+                            kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        if (a.Tw > 0) {
+            if (!encode_tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.win, kD, (uint64_t)(a.B * a.Tw), kD * 2, 64,
+                                kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        } else {
+            mw = mc;
+        }
+    } else {
+        mc = mq;   // unused by the FP8 kernel
+        mw = mq;
+    }
+    auto kern = (a.kv_dtype == LCS_KV_FP8) ? attend_tc_kernel<true> : attend_tc_kernel<false>;
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), kAtSmem);
+    if (e != cudaSuccess) return e;
+    const int splits = choose_splits(a);
     float* part_o = nullptr;
     float* part_ml = nullptr;
     if (splits > 1) {
         part_o = static_cast<float*>(scratch);
         part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256(queries * splits * kH * kDv * 4));
     }
-    auto kern = (a.kv_dtype == LCS_KV_FP8) ? attend_tc_kernel<true> : attend_tc_kernel<false>;
-    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), kAtSmem);
-    if (e != cudaSuccess) return e;
-    e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, a, splits, part_o,
-                 part_ml, status);
-    if (e != cudaSuccess || splits == 1) return e;
-    attend_combine_kernel<<<(unsigned)(queries * kH), 128, 0, s>>>(part_o, part_ml, splits, a.out, a.out_dtype,
-                                                                    a.lse);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(queries * splits));
+    cfg.blockDim = dim3(kAtThreads);
+    cfg.dynamicSmemBytes = kAtSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)splits;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kern, mq, mc, mw, a, splits, part_o, part_ml, status);
 }
 
 }  // namespace lcs

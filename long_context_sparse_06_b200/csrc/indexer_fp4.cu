@@ -18,15 +18,16 @@
 //  * E_{h,b} * sk_{s,b} equals D_b * sq_{h,b} * sk_{s,b} exactly, so the epilogue
 //    fma(E, sk, acc) chain reproduces the fma(D, sq*sk, acc) chain bit for bit.
 //
-// Kernel layout (persistent, one CTA per SM, 320 threads):
+// Kernel layout (persistent, one CTA per SM, 448 threads):
 //   warp 0     TMA: packed key tiles [128 keys x 64 B] into a 6-stage raw ring, and
 //              the group's dequantised query heads [64 x 128 bf16] into one of 2 slots
 //   warp 1     tcgen05.mma (M = 128 keys, N = 64 heads, K = 32 per block) into one of
 //              two 256-column accumulator sets (4 blocks x 64 heads)
 //   warps 2-5  converters: one key row per thread, packed bytes -> bf16 codes through a
 //              lane-replicated 256-entry table, into a 3-stage 128-byte-swizzled ring
-//   warps 6-9  epilogue: one key row per thread, block/heads combine, ReLU-weighted head
-//              chain, bf16 score
+//   warps 6-13 epilogue, two groups of 4 warps taking alternate tiles (one accumulator
+//              set each): one key row per thread, block/heads combine, ReLU-weighted
+//              head chain, bf16 score
 #include <utility>
 
 #include "lcs_common.cuh"
@@ -42,7 +43,7 @@ constexpr int kRawTile = kBM * kDI / 2;           // 8 KB packed
 constexpr int kATile = kBM * kDI * 2;             // 32 KB bf16
 constexpr int kBTile = kHeads * kDI * 2;          // 16 KB bf16
 constexpr int kLutBytes = 256 * 32 * 4;           // byte -> 2 bf16, one copy per lane
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr size_t kSmem = 1024 + kAStages * kATile + 2 * kBTile + kRawStages * kRawTile + kLutBytes;
 
 struct Bars {
@@ -211,7 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4* src = reinterpret_cast<const uint4*>(raw + rs * kRawTile + row * 64);
             uint8_t* dst = a_tiles + as * kATile;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {            // 32 codes per 16 bytes
+            for (int qq = 0; qq < 4; ++qq) {         // 32 codes per 16 bytes
+                // rows 64 B apart: rotating the piece order by row/2 keeps the 8 rows of a
+                // shared-memory phase on distinct banks
+                const int q = (qq + (row >> 1)) & 3;
                 const uint4 v = src[q];
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
                 uint32_t o[16];
@@ -232,50 +236,84 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_it;
         }
     } else {
-        // ---------------- epilogue: warps 6..9, TMEM lane quarter = warp % 4, thread = key row
+        // ---------------- epilogue: warps 6..13 in two groups of 4 (group e takes the tiles
+        // with n_it % 2 == e, i.e. accumulator set e); TMEM lane quarter = warp % 4, thread =
+        // key row.
+        const int e = (warp - 6) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        int64_t prev_g = -1, n_it = 0;
-        float wr[kHeads];
-        for (int64_t it = it0; it < it1; ++it) {
+        int64_t n_it = 0;
+        // The key scales of a tile are loaded two of this group's tiles early, so that
+        // their global-load latency overlaps the combine of the tiles in between.
+        constexpr int kSkAhead = 2;
+        auto load_sk = [&](int64_t i) -> uint32_t {
+            if (i >= it1) return 0u;
+            const int64_t gg = i / tiles_per, ss = (i - gg * tiles_per) * kBM + row;
+            return ss < N_c ? __ldg(reinterpret_cast<const uint32_t*>(k_scales + ((gg / Q) * N_c + ss) * 4)) : 0u;
+        };
+        // tiles of this group: the valid tiles (tile * kBM < avail) with n_it % 2 == e
+        int64_t next_it[kSkAhead + 1];
+        uint32_t skq[kSkAhead];
+        auto advance = [&](int64_t from, int64_t& cnt) -> int64_t {   // next tile of group e
+            for (int64_t i = from; i < it1; ++i) {
+                const int64_t gg = i / tiles_per, tt = i - gg * tiles_per;
+                if (tt * kBM >= avail(q_pos, gg, m, N_c)) continue;
+                const int64_t c = cnt++;
+                if ((c & 1) == e) return i;
+            }
+            return it1;
+        };
+        int64_t cnt = 0;
+        next_it[0] = advance(it0, cnt);
+#pragma unroll
+        for (int i = 1; i <= kSkAhead; ++i) next_it[i] = advance(next_it[i - 1] + 1, cnt);
+#pragma unroll
+        for (int i = 0; i < kSkAhead; ++i) skq[i] = load_sk(next_it[i]);
+        while (next_it[0] < it1) {
+            const int64_t it = next_it[0];
+            const uint32_t skw = skq[0];
+#pragma unroll
+            for (int i = 0; i < kSkAhead; ++i) next_it[i] = next_it[i + 1];
+            next_it[kSkAhead] = advance(next_it[kSkAhead - 1] + 1, cnt);
+#pragma unroll
+            for (int i = 0; i + 1 < kSkAhead; ++i) skq[i] = skq[i + 1];
+            skq[kSkAhead - 1] = load_sk(next_it[kSkAhead - 1]);
             const int64_t g = it / tiles_per, tile = it - g * tiles_per;
             const int64_t n = avail(q_pos, g, m, N_c);
-            if (tile * kBM >= n) continue;
-            if (g != prev_g) {
-#pragma unroll
-                for (int h = 0; h < kHeads; ++h) wr[h] = __ldg(w + g * kHeads + h);
-                prev_g = g;
-            }
+            const float4* wg4 = reinterpret_cast<const float4*>(w + g * kHeads);   // L1-resident
             const int64_t s = tile * kBM + row;
-            const int64_t b = g / Q;
-            uint32_t skw = 0;
-            if (s < N_c) skw = __ldg(reinterpret_cast<const uint32_t*>(k_scales + (b * N_c + s) * 4));
             float sk[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) sk[i] = e4m3_to_f32((uint8_t)(skw >> (8 * i)));
-            const int cb = (int)(n_it & 1);
-            if (!mbar_wait(&bars.cfull[cb], (uint32_t)((n_it >> 1) & 1), status, 118)) break;
+            // the k-th tile of this group is the k-th use of accumulator set e
+            if (!mbar_wait(&bars.cfull[e], (uint32_t)(n_it & 1), status, 118)) break;
             tc_fence_after();
             float acc = 0.f;
 #pragma unroll
             for (int h0 = 0; h0 < kHeads; h0 += 16) {
-                uint32_t e[4][16];
+                uint32_t ev[4][16];
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk)
-                    tmem_ld16(tmem_addr(tmem, quarter * 32, cb * 256 + blk * 64 + h0), e[blk]);
+                    tmem_ld16(tmem_addr(tmem, quarter * 32, e * 256 + blk * 64 + h0), ev[blk]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float dot = __uint_as_float(e[0][j]) * sk[0];
-                    dot = fmaf(__uint_as_float(e[1][j]), sk[1], dot);
-                    dot = fmaf(__uint_as_float(e[2][j]), sk[2], dot);
-                    dot = fmaf(__uint_as_float(e[3][j]), sk[3], dot);
-                    acc = fmaf(wr[h0 + j], dot > 0.f ? dot : 0.f, acc);
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    const float4 w4 = __ldg(wg4 + h0 / 4 + j4);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * j4 + jj;
+                        float dot = __uint_as_float(ev[0][j]) * sk[0];
+                        dot = fmaf(__uint_as_float(ev[1][j]), sk[1], dot);
+                        dot = fmaf(__uint_as_float(ev[2][j]), sk[2], dot);
+                        dot = fmaf(__uint_as_float(ev[3][j]), sk[3], dot);
+                        acc = fmaf(wv[jj], dot > 0.f ? dot : 0.f, acc);
+                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.cempty[cb]);
+            if (lane == 0) mbar_arrive(&bars.cempty[e]);
             if (s < N_c) scores[g * N_c + s] = (s < n) ? f32_to_bf16_bits(acc) : (uint16_t)0xFF80u;   // -inf
             ++n_it;
         }

@@ -240,6 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
 
 #if defined(__CUDA_ARCH__)
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // The dependent kernel (attention) may start its prologue now: it reads this kernel's
+    // output only after its own griddepcontrol.wait, which waits for this grid to finish.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #endif
 
     if (n <= k) {

@@ -296,18 +296,20 @@ def test_hca_attend_decode_tc(L, orc):
         assert_close_abs(lse[b, 0], l, 2e-2, f"hca lse b {b}")
 
 
-def test_attend_prefill_tc_causal(L, orc):
-    """C4-shaped (smaller): queries at positions p0.., window from the chunk plus a 127-row prefix tail."""
+@pytest.mark.parametrize("tail", [127, 50])
+def test_attend_prefill_tc_causal(L, orc, tail):
+    """C4-shaped (smaller): queries at positions p0.., window from the chunk plus a prefix tail
+    of `tail` raw rows (50: the first queries see partial windows of 51.. rows)."""
     B, Q, H, D, dv, k, W = 1, 24, 64, 576, 512, 256, 128
     p0 = 4000
     Nc = (p0 + Q) // 4
-    Tw = 127 + Q
+    Tw = tail + Q
     scale = 1 / math.sqrt(576)
     q = randn("g.ap.q", (B, Q, H, D), dtype=torch.bfloat16)
     comp = randn("g.ap.c", (B, Nc, D), dtype=torch.bfloat16)
     win = randn("g.ap.w", (B, Tw, D), dtype=torch.bfloat16)
     q_pos = (p0 + torch.arange(Q, dtype=torch.int64)).reshape(B, Q)
-    wp0 = torch.tensor([p0 - 127], dtype=torch.int64)
+    wp0 = torch.tensor([p0 - tail], dtype=torch.int64)
     nav = [[orc.n_avail(int(t), 4, Nc) for t in q_pos[0]]]
     idx = _rand_sel("sel.pf", B, Q, k, nav)
     out = both_outputs(lambda od: L.csa_attend(q.to(DEV), comp.to(DEV), win.to(DEV), torch.from_numpy(idx).to(DEV),
@@ -315,7 +317,7 @@ def test_attend_prefill_tc_causal(L, orc):
                                                out_dtype=od)).cpu().numpy()
     for t in range(Q):
         o, _ = orc.csa_attend(q[0, t].double().numpy(), comp[0].double().numpy(), idx[0, t],
-                              win[0].double().numpy(), p0 - 127, int(q_pos[0, t]), W, dv, scale)
+                              win[0].double().numpy(), p0 - tail, int(q_pos[0, t]), W, dv, scale)
         assert_close_rel_rms(out[0, t], o, 2e-2, f"prefill q {t}")
     # HCA causal with m' = 128 on the same queries
     Nh = (p0 + Q) // 128
@@ -324,7 +326,7 @@ def test_attend_prefill_tc_causal(L, orc):
                                                 out_dtype=od)).cpu().numpy()
     for t in range(0, Q, 5):
         o, _ = orc.hca_attend(q[0, t].double().numpy(), comp[0, :Nh].double().numpy(), 128, win[0].double().numpy(),
-                              p0 - 127, int(q_pos[0, t]), W, dv, scale)
+                              p0 - tail, int(q_pos[0, t]), W, dv, scale)
         assert_close_rel_rms(outh[0, t], o, 2e-2, f"hca prefill q {t}")
 
 
