@@ -186,15 +186,15 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     const uint32_t tmem = bars.tmem_base;
 
     // ---- what does not depend on the preceding kernel: the window rows, which fill the
-    // first chunks of the row list (the last one padded), the chunk range of this split
-    // (planned for the longest selection), Q.
+    // first chunks of the row list (the last one padded), and Q.
     const WinPlan wp = plan_window(a, g);
     const int64_t nwc = (wp.nwin + kChunk - 1) / kChunk;
     const int64_t comp_max = (a.idx != nullptr) ? a.k : hca_avail(a, g);
     const int64_t nch_max = nwc + (comp_max + kChunk - 1) / kChunk;
-    const int64_t cps = (nch_max + splits - 1) / splits;
-    const int64_t c_begin = sp * cps;
-    const bool q_wanted = c_begin < nch_max;
+    // chunks are dealt to the splits round-robin: local chunk c is global chunk sp + splits*c
+    // (the window chunks, loaded by TMA, and the gathered ones spread over the splits)
+    auto gcof = [&](int c) -> int64_t { return sp + (int64_t)splits * c; };
+    const bool q_wanted = sp < nch_max;
     if (warp == kWarpQK && lane == 0 && q_wanted) {
         mbar_arrive_expect_tx(&bars.qfull, kQBytes);
         for (int blk = 0; blk < 9; ++blk)
@@ -304,8 +304,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // wait for the preceding kernel when it is a window chunk of this split.
     bool pre = false;
     if (producer) {
-        const int64_t gc = c_begin + pst;
-        if (pst < cps && gc < nch_max && gc < nwc) {
+        const int64_t gc = gcof(pst);
+        if (gc < nwc) {
             fill(gc, my_row_src(gc));
             pre = true;
         }
@@ -343,8 +343,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     __syncthreads();
     nsel = bars.nsel;
     const int64_t nch_all = nwc + (nsel + kChunk - 1) / kChunk;
-    const int64_t c_end = (c_begin + cps < nch_all) ? c_begin + cps : nch_all;
-    const int nch = (int)(c_end > c_begin ? c_end - c_begin : 0);
+    const int nch = sp < nch_all ? (int)((nch_all - sp + splits - 1) / splits) : 0;
 
     constexpr uint32_t idesc_qk = idesc_bf16(64, kChunk, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16(64, 256, false, true);
@@ -404,13 +403,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         // ---------------- producer loop (the group's chunks pst, pst+2, ...); a stage is
         // refilled once the P.V that read it is complete.  The next chunk's row sources are
         // resolved while this chunk's copies are in flight.
-        const uint8_t* nxt = (pst < nch) ? my_row_src(c_begin + pst) : nullptr;
+        const uint8_t* nxt = (pst < nch) ? my_row_src(gcof(pst)) : nullptr;
         for (int c = pst; c < nch; c += 2) {
             const uint8_t* my_src = nxt;
             const int u = c >> 1;
             if (u >= 1 && !mbar_wait(&bars.kempty[pst], (uint32_t)((u - 1) & 1), status, 310)) break;
-            if (c + 2 < nch) nxt = my_row_src(c_begin + c + 2);
-            if (!(pre && c == pst)) fill(c_begin + c, my_src);
+            if (c + 2 < nch) nxt = my_row_src(gcof(c + 2));
+            if (!(pre && c == pst)) fill(gcof(c), my_src);
         }
     } else if (warp < 4) {
         // ---------------- softmax / correction / epilogue: warps 0..3.  Warp q owns heads
@@ -432,7 +431,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&bars.sempty[st]);
-            const int nvalid = chunk_valid(c_begin + c);
+            const int nvalid = chunk_valid(gcof(c));
             float mx = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 32; ++j)

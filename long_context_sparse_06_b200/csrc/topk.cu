@@ -188,36 +188,62 @@ __device__ void find_bin(TopkSmem& sm, uint32_t k) {
     __syncthreads();
 }
 
-// Loads the 32 consecutive keys [i0, i0+32) of lane-owned scores (clipped at n).
+// One warp batch of 1024 keys starting at bb, loaded coalesced: lane l holds the kE keys
+// bb + 32*kE*v + kE*l + j (v < kV, j < kE).  A whole batch of a 16-byte aligned row is
+// kV 16-byte loads per lane, all issued before any is used (raw words, converted to keys
+// later, so that the next batch's loads can be in flight while this one is processed);
+// a partial batch or an unaligned row uses element loads, keys at or beyond n invalid.
 template <bool BF16>
-__device__ __forceinline__ void load32(const char* srow, int64_t i0, int64_t n, uint32_t (&key)[32]) {
-    if (i0 + 32 <= n) {
-        if constexpr (BF16) {
-            const uint4* p = reinterpret_cast<const uint4*>(srow + i0 * 2);
+struct Batch {
+    static constexpr int kE = BF16 ? 8 : 4, kV = 1024 / (32 * kE);
+    uint4 raw[kV];
+    bool whole;
+};
+template <bool BF16>
+__device__ __forceinline__ void issue_batch(const char* srow, bool vec_ok, int64_t bb, int64_t n, int lane,
+                                            Batch<BF16>& bt) {
+    constexpr int kE = Batch<BF16>::kE, kV = Batch<BF16>::kV;
+    bt.whole = vec_ok && bb + 1024 <= n;
+    if (bt.whole) {
+        const uint4* p = reinterpret_cast<const uint4*>(srow + (bb + kE * lane) * (BF16 ? 2 : 4));
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const uint4 w = __ldg(p + v);
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int v = 0; v < kV; ++v) bt.raw[v] = __ldg(p + v * 32);
+    }
+}
+// Keys of a batch (and the valid mask per vector slot).
+template <bool BF16>
+__device__ __forceinline__ void batch_keys(const char* srow, int64_t bb, int64_t n, int lane, const Batch<BF16>& bt,
+                                           uint32_t (&key)[Batch<BF16>::kV][Batch<BF16>::kE],
+                                           uint32_t (&valid)[Batch<BF16>::kV]) {
+    constexpr int kE = Batch<BF16>::kE, kV = Batch<BF16>::kV;
+    if (bt.whole) {
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            valid[v] = (1u << kE) - 1u;
+            const uint32_t ww[4] = {bt.raw[v].x, bt.raw[v].y, bt.raw[v].z, bt.raw[v].w};
+            if constexpr (BF16) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    key[8 * v + 2 * q] = bf16_key((uint16_t)(ww[q] & 0xFFFF));
-                    key[8 * v + 2 * q + 1] = bf16_key((uint16_t)(ww[q] >> 16));
+                    key[v][2 * q] = bf16_key((uint16_t)(ww[q] & 0xFFFF));
+                    key[v][2 * q + 1] = bf16_key((uint16_t)(ww[q] >> 16));
                 }
-            }
-        } else {
-            const float4* p = reinterpret_cast<const float4*>(srow + i0 * 4);
+            } else {
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                const float4 f = __ldg(p + v);
-                key[4 * v] = f32_key(f.x);
-                key[4 * v + 1] = f32_key(f.y);
-                key[4 * v + 2] = f32_key(f.z);
-                key[4 * v + 3] = f32_key(f.w);
+                for (int q = 0; q < 4; ++q) key[v][q] = f32_key(__uint_as_float(ww[q]));
             }
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) key[j] = (i0 + j < n) ? load_key<BF16>(srow, i0 + j) : 0u;
+        for (int v = 0; v < kV; ++v) {
+            const int64_t i = bb + 32 * kE * v + kE * lane;
+            valid[v] = 0;
+#pragma unroll
+            for (int j = 0; j < kE; ++j) {
+                const bool ok = i + j < n;
+                key[v][j] = ok ? load_key<BF16>(srow, i + j) : 0u;
+                valid[v] |= (ok ? 1u : 0u) << j;
+            }
+        }
     }
 }
 
@@ -264,34 +290,62 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
         for (int i = t; i < kBins + kBins / 32; i += kThreads) sm.bins[i] = 0;
     }
 
-    // ---- 2. one pass: lane-owned runs of 32 consecutive keys; keys >= T go to the warp's
-    // buffer in index order (per-lane counts, warp scan for the lane's slot base)
+    // ---- 2. one pass over the row: warp w owns [w0, w1) in whole batches of 1024 keys,
+    // loaded coalesced, the next batch in flight (see issue_batch).  Keys >= T go to the warp's buffer in index order:
+    // a key's slot is the warp's running count, plus the batch counts of the earlier
+    // load slots v, plus the counts of the lower lanes in slot v (a warp prefix sum of
+    // the per-slot counts packed in 16-bit fields), plus the earlier keys of its own vector.
     unsigned long long* wb = sm.wbuf + warp * kWarpCap;
-    const int64_t per_warp = ((n + kWarps - 1) / kWarps + 1023) / 1024 * 1024;   // whole 32x32 batches
+    const int64_t per_warp = ((n + kWarps - 1) / kWarps + 1023) / 1024 * 1024;
     const int64_t w0 = warp * per_warp, w1 = (w0 + per_warp < n) ? w0 + per_warp : n;
+    const bool vec_ok = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
+    constexpr int kE = Batch<BF16>::kE, kV = Batch<BF16>::kV;
     uint32_t wcnt = 0;
+    Batch<BF16> nb;
+    if (w0 < w1) issue_batch<BF16>(srow, vec_ok, w0, w1, lane, nb);
     for (int64_t bb = w0; bb < w1; bb += 1024) {
-        const int64_t i0 = bb + 32 * lane;
-        uint32_t key[32];
-        load32<BF16>(srow, i0, w1, key);
-        uint32_t c = 0;
+        uint32_t key[kV][kE], valid[kV];
+        batch_keys<BF16>(srow, bb, w1, lane, nb, key, valid);
+        if (bb + 1024 < w1) issue_batch<BF16>(srow, vec_ok, bb + 1024, w1, lane, nb);
+        uint32_t pm[kV], cnt[kV];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) c += (i0 + j < w1 && key[j] >= T);
-        uint32_t incl = c;
+        for (int v = 0; v < kV; ++v) {
+            pm[v] = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += x;
+            for (int j = 0; j < kE; ++j) pm[v] |= (key[v][j] >= T ? 1u : 0u) << j;
+            pm[v] &= valid[v];
+            cnt[v] = __popc(pm[v]);
         }
-        uint32_t slot = wcnt + incl - c;
+        uint32_t incl[kV / 2], tot[kV / 2];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (i0 + j < w1 && key[j] >= T) {
-                if (slot < kWarpCap)
-                    wb[slot] = ((unsigned long long)key[j] << 32) | (unsigned long long)(~(uint32_t)(i0 + j));
-                ++slot;
+        for (int w = 0; w < kV / 2; ++w) {
+            const uint32_t own = cnt[2 * w] | (cnt[2 * w + 1] << 16);
+            uint32_t x = own;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
             }
-        wcnt += __shfl_sync(0xffffffffu, incl, 31);
+            tot[w] = __shfl_sync(0xffffffffu, x, 31);
+            incl[w] = x - own;   // exclusive
+        }
+        uint32_t base = wcnt;
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            const uint32_t ex = (v & 1) ? (incl[v >> 1] >> 16) : (incl[v >> 1] & 0xFFFF);
+            const uint32_t tv = (v & 1) ? (tot[v >> 1] >> 16) : (tot[v >> 1] & 0xFFFF);
+            uint32_t slot = base + ex;
+            const int64_t i = bb + 32 * kE * v + kE * lane;
+#pragma unroll
+            for (int j = 0; j < kE; ++j)
+                if ((pm[v] >> j) & 1u) {
+                    if (slot < kWarpCap)
+                        wb[slot] = ((unsigned long long)key[v][j] << 32) | (unsigned long long)(~(uint32_t)(i + j));
+                    ++slot;
+                }
+            base += tv;
+        }
+        wcnt = base;
     }
     if (lane == 0) { sm.warp_cnt[warp] = wcnt; sm.wsum[warp] = wcnt; }
     __syncthreads();

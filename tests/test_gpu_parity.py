@@ -107,8 +107,9 @@ def test_compress(L, orc, case):
 
 # --------------------------------------------------------------------- top-k
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_topk_bit_exact_on_same_scores(L, orc, dtype):
-    rows, N = 7, 3000
+@pytest.mark.parametrize("N", [3000, 2999])   # 2999: rows after the first start off 16-byte alignment
+def test_topk_bit_exact_on_same_scores(L, orc, dtype, N):
+    rows = 7
     s = randn("g.tk", (1, rows, N), std=4.0)
     s[0, 1] = torch.round(s[0, 1])                 # heavy ties
     s[0, 2] = 0.0
