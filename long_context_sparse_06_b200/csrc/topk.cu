@@ -45,6 +45,8 @@ constexpr int kBins = 1 << kBinBits;
 constexpr int kCandCap = 2048;                 // threshold-bin elements ranked by counting
 constexpr int kWarpCap = 512;                  // per-warp candidate buffer
 constexpr int kListCap = kWarps * kWarpCap;    // all candidates
+constexpr int kMaxP = 16;                      // CTAs per row (one cluster)
+static_assert(kMaxP <= kWarps, "per-rank counts reuse the per-warp arrays");
 
 struct TopkSmem {
     uint32_t bins[kBins + kBins / 32];          // 64 KB histogram, one pad word per 32 bins
@@ -250,11 +252,12 @@ __device__ __forceinline__ void batch_keys(const char* srow, int64_t bb, int64_t
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restrict__ scores, int64_t N_c,
                                                            const int64_t* __restrict__ q_pos, int m, int k,
-                                                           int32_t* __restrict__ idx_out) {
+                                                           int32_t* __restrict__ idx_out, int P) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     constexpr int kShift = (BF16 ? 16 : 32) - kBinBits;
-    const int64_t row = blockIdx.x;
+    const int64_t row = blockIdx.x / P;
+    const int rank = (int)(blockIdx.x - row * P);   // == rank in the row's cluster
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     int64_t n = N_c;
     if (q_pos != nullptr) {
@@ -296,8 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
     // load slots v, plus the counts of the lower lanes in slot v (a warp prefix sum of
     // the per-slot counts packed in 16-bit fields), plus the earlier keys of its own vector.
     unsigned long long* wb = sm.wbuf + warp * kWarpCap;
-    const int64_t per_warp = ((n + kWarps - 1) / kWarps + 1023) / 1024 * 1024;
-    const int64_t w0 = warp * per_warp, w1 = (w0 + per_warp < n) ? w0 + per_warp : n;
+    const int64_t part = ((n + P - 1) / P + 1023) / 1024 * 1024;   // this CTA's part of the row
+    const int64_t r0 = rank * part, r1 = (r0 + part < n) ? r0 + part : n;
+    const int64_t per_warp = ((r1 > r0 ? r1 - r0 : 0) + kWarps * 1024 - 1) / (kWarps * 1024) * 1024;
+    const int64_t w0 = r0 + warp * per_warp, w1 = (w0 + per_warp < r1) ? w0 + per_warp : r1;
     const bool vec_ok = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
     constexpr int kE = Batch<BF16>::kE, kV = Batch<BF16>::kV;
     uint32_t wcnt = 0;
@@ -351,21 +356,76 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
     __syncthreads();
     scan_warp_sums(sm);
     if (t == 0) {
-        uint32_t fail = sm.total < (uint32_t)k;
+        uint32_t fail = (P == 1) && sm.total < (uint32_t)k;
         for (int w = 0; w < kWarps; ++w) fail |= sm.warp_cnt[w] > (uint32_t)kWarpCap;
         sm.fail = fail;
     }
     __syncthreads();
-    if (sm.fail) {
+    if (P == 1 && sm.fail) {
         radix_select<BF16>(sm, srow, n, k, out);
         return;
     }
-    const uint32_t C = sm.total;
-    {
+    if (!sm.fail) {
         const uint32_t o = sm.wsum[warp];
         for (uint32_t j = lane; j < wcnt; j += 32) sm.list[o + j] = wb[j];
     }
     __syncthreads();
+    if (P > 1) {
+        // ---- the row's CTAs form one cluster: CTA 0 appends the peers' candidate lists
+        // (slices in rank order, so the list stays in index order) through distributed
+        // shared memory, then selects; a missed bound falls back to CTA 0 alone.
+        cluster_sync_all();
+        if (rank == 0) {
+            if (t < 32) {   // lane r reads rank r's count and flag (one remote load each, in parallel)
+                const bool has = t < P;
+                const uint32_t c = has ? ld_dsmem_u32(dsmem_addr(&sm.total, (uint32_t)t)) : 0u;
+                const uint32_t f = has ? ld_dsmem_u32(dsmem_addr(&sm.fail, (uint32_t)t)) : 0u;
+                uint32_t incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (t >= o) incl += y;
+                }
+                const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+                const bool anyf = __any_sync(0xffffffffu, f != 0);
+                __syncwarp();
+                if (has) {
+                    sm.warp_off[t] = incl - c;
+                    sm.warp_cnt[t] = c;
+                }
+                if (t == 0) {
+                    sm.fail = anyf || tot < (uint32_t)k || tot > (uint32_t)kListCap;
+                    sm.total = tot;
+                }
+            }
+            __syncthreads();
+            if (!sm.fail)
+                for (int r = 1; r < P; ++r) {   // four remote loads in flight per thread
+                    const uint32_t c = sm.warp_cnt[r], o = sm.warp_off[r];
+                    const uint32_t src = dsmem_addr(&sm.list[0], (uint32_t)r);
+                    for (uint32_t j0 = t; j0 < c; j0 += 4 * kThreads) {
+                        unsigned long long v[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t j = j0 + u * kThreads;
+                            v[u] = j < c ? ld_dsmem_u64(src + j * 8) : 0ull;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t j = j0 + u * kThreads;
+                            if (j < c) sm.list[o + j] = v[u];
+                        }
+                    }
+                }
+        }
+        cluster_sync_all();   // the peers' lists have been read
+        if (rank != 0) return;
+        if (sm.fail) {
+            radix_select<BF16>(sm, srow, n, k, out);
+            return;
+        }
+    }
+    const uint32_t C = sm.total;
 
     // ---- 3. exact selection among the candidates
     for (uint32_t j = t; j < C; j += kThreads) atomicAdd(&sm.bins[hb((uint32_t)(sm.list[j] >> 32) >> kShift)], 1u);
@@ -439,6 +499,74 @@ int64_t topk_scratch_bytes(int64_t rows, int64_t N_c) {
     return 0;
 }
 
+namespace {
+// CTAs per row: enough to spread the row pass over the SMs for a few rows, each CTA taking
+// at least 4096 keys; one cluster per row, resident all at once.
+template <bool BF16>
+int choose_ranks(int64_t rows, int64_t N_c) {
+    int64_t p = num_sms() / (rows > 0 ? rows : 1);
+    const int64_t by_len = (N_c + 4095) / 4096;
+    if (p > by_len) p = by_len;
+    if (p > kMaxP) p = kMaxP;
+    static std::mutex mu;
+    static int cache[kMaxP + 1];
+    std::lock_guard<std::mutex> lock(mu);
+    const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16>);
+    for (; p > 1; --p) {
+        if (cache[p] == 0) {
+            int n = 0;
+            if (p <= 8 || cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+                cudaLaunchConfig_t cfg = {};
+                cfg.gridDim = dim3((unsigned)p);
+                cfg.blockDim = dim3(kThreads);
+                cfg.dynamicSmemBytes = sizeof(TopkSmem);
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = (unsigned)p;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+            }
+            cudaGetLastError();
+            cache[p] = n > 0 ? n : -1;
+        }
+        if (cache[p] >= rows) break;
+    }
+    return (int)(p < 1 ? 1 : p);
+}
+
+template <bool BF16>
+cudaError_t launch_topk_t(const void* scores, int64_t rows, int64_t N_c, const int64_t* q_pos, int m, int k,
+                          int32_t* idx, cudaStream_t s, bool pdl) {
+    const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16>);
+    cudaError_t e = set_smem_once(kern, sizeof(TopkSmem));
+    if (e != cudaSuccess) return e;
+    const int P = choose_ranks<BF16>(rows, N_c);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * P));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sizeof(TopkSmem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)P;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, topk_kernel<BF16>, scores, N_c, q_pos, m, k, idx, P);
+}
+}  // namespace
+
 cudaError_t launch_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, int64_t N_c,
                         const int64_t* q_pos, int m, int k, int32_t* idx, void* scratch, int* status,
                         cudaStream_t s, bool pdl) {
@@ -446,17 +574,8 @@ cudaError_t launch_topk(const void* scores, int score_dtype, int64_t B, int64_t 
     (void)status;
     const int64_t rows = B * Q;
     if (rows == 0 || k == 0) return cudaSuccess;
-    const size_t smem = sizeof(TopkSmem);
-    if (score_dtype == LCS_BF16) {
-        cudaError_t e = set_smem_once(reinterpret_cast<const void*>(topk_kernel<true>), smem);
-        if (e != cudaSuccess) return e;
-        return launch_k(topk_kernel<true>, dim3((unsigned)rows), dim3(kThreads), smem, s, pdl, scores, N_c, q_pos, m,
-                        k, idx);
-    }
-    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(topk_kernel<false>), smem);
-    if (e != cudaSuccess) return e;
-    return launch_k(topk_kernel<false>, dim3((unsigned)rows), dim3(kThreads), smem, s, pdl, scores, N_c, q_pos, m, k,
-                    idx);
+    return score_dtype == LCS_BF16 ? launch_topk_t<true>(scores, rows, N_c, q_pos, m, k, idx, s, pdl)
+                                   : launch_topk_t<false>(scores, rows, N_c, q_pos, m, k, idx, s, pdl);
 }
 
 }  // namespace lcs
