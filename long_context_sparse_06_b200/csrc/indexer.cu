@@ -124,8 +124,9 @@ __global__ void __launch_bounds__(kIxThreads, 1)
         if (lane == 0) {
             // ---------------- TMA producer
             int64_t prev_g = -1, gseq = -1, n_it = 0;
-            for (int64_t it = it0; it < it1; ++it) {
-                const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+            TileIt ti(it0, (int)tiles_per, (int)Q);
+            for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
+                const int64_t g = ti.g, tile = ti.tile;
                 if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
                 if (g != prev_g) {
                     ++gseq;
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(kIxThreads, 1)
                 const int st = (int)(n_it % kStages);
                 if (!mbar_wait(&bars.empty[st], (uint32_t)(((n_it / kStages) & 1) ^ 1), status, 102)) break;
                 mbar_arrive_expect_tx(&bars.full[st], kATile);
-                const int64_t b = g / Q;
+                const int64_t b = ti.b;
                 for (int kb = 0; kb < 2; ++kb)
                     tma_load_2d(a_tiles + st * kATile + kb * (kATile / 2), &map_k, &bars.full[st], kb * 64,
                                 (int)(b * N_c + tile * kBM));
@@ -154,8 +155,9 @@ __global__ void __launch_bounds__(kIxThreads, 1)
             int64_t prev_g = -1, gseq = -1, n_it = 0;
             int slot = 0;
             bool ok = true;
-            for (int64_t it = it0; it < it1 && ok; ++it) {
-                const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+            TileIt ti(it0, (int)tiles_per, (int)Q);
+            for (int64_t it = it0; it < it1 && ok; ++it, ti.next((int)tiles_per, (int)Q)) {
+                const int64_t g = ti.g, tile = ti.tile;
                 if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
                 if (g != prev_g) {
                     if (prev_g >= 0) mma_commit(&bars.bempty[slot]);   // previous group's heads are free
@@ -191,8 +193,9 @@ __global__ void __launch_bounds__(kIxThreads, 1)
         const int row = quarter * 32 + lane;
         int64_t prev_g = -1, n_it = 0;
         float wr[kHeads];
-        for (int64_t it = it0; it < it1; ++it) {
-            const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+        TileIt ti(it0, (int)tiles_per, (int)Q);
+        for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
+            const int64_t g = ti.g, tile = ti.tile;
             const int64_t n = avail(q_pos, g, m, N_c);
             if (tile * kBM >= n) continue;
             if (g != prev_g) {

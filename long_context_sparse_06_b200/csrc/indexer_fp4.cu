@@ -138,8 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             // ---------------- TMA producer
             int64_t prev_g = -1, gseq = -1, n_it = 0;
-            for (int64_t it = it0; it < it1; ++it) {
-                const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+            TileIt ti(it0, (int)tiles_per, (int)Q);
+            for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
+                const int64_t g = ti.g, tile = ti.tile;
                 if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
                 if (g != prev_g) {
                     ++gseq;
@@ -154,8 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int rs = (int)(n_it % kRawStages);
                 if (!mbar_wait(&bars.rempty[rs], (uint32_t)(((n_it / kRawStages) & 1) ^ 1), status, 112)) break;
                 mbar_arrive_expect_tx(&bars.rfull[rs], kRawTile);
-                const int64_t b = g / Q;
-                tma_load_2d(raw + rs * kRawTile, &map_k, &bars.rfull[rs], 0, (int)(b * N_c + tile * kBM));
+                tma_load_2d(raw + rs * kRawTile, &map_k, &bars.rfull[rs], 0, (int)(ti.b * N_c + tile * kBM));
                 ++n_it;
             }
         }
@@ -167,8 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t b_desc0 = sw128_desc(smem_u32(b_tiles), 16, 1024);
             int64_t prev_g = -1, gseq = -1, n_it = 0;
             int slot = 0;
-            for (int64_t it = it0; it < it1; ++it) {
-                const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+            TileIt ti(it0, (int)tiles_per, (int)Q);
+            for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
+                const int64_t g = ti.g, tile = ti.tile;
                 if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
                 if (g != prev_g) {
                     if (prev_g >= 0) mma_commit(&bars.bempty[slot]);
@@ -203,9 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- converters: thread = key row of the tile
         const int row = threadIdx.x - 64;
         int64_t n_it = 0;
-        for (int64_t it = it0; it < it1; ++it) {
-            const int64_t g = it / tiles_per, tile = it - g * tiles_per;
-            if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
+        TileIt ti(it0, (int)tiles_per, (int)Q);
+        for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
+            if (ti.tile * kBM >= avail(q_pos, ti.g, m, N_c)) continue;
             const int rs = (int)(n_it % kRawStages), as = (int)(n_it % kAStages);
             if (!mbar_wait(&bars.rfull[rs], (uint32_t)((n_it / kRawStages) & 1), status, 116)) break;
             if (!mbar_wait(&bars.aempty[as], (uint32_t)(((n_it / kAStages) & 1) ^ 1), status, 117)) break;
@@ -242,44 +243,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int e = (warp - 6) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        int64_t n_it = 0;
-        // The key scales of a tile are loaded two of this group's tiles early, so that
-        // their global-load latency overlaps the combine of the tiles in between.
-        constexpr int kSkAhead = 2;
-        auto load_sk = [&](int64_t i) -> uint32_t {
-            if (i >= it1) return 0u;
-            const int64_t gg = i / tiles_per, ss = (i - gg * tiles_per) * kBM + row;
-            return ss < N_c ? __ldg(reinterpret_cast<const uint32_t*>(k_scales + ((gg / Q) * N_c + ss) * 4)) : 0u;
+        int64_t n_it = 0;   // tiles of this group so far
+        // The key scales of this group's tile are prefetched two of its tiles early (tile
+        // it + 4 of the sequence, when no tile is skipped); a mismatch loads them directly.
+        auto load_sk = [&](int64_t b, int64_t tile) -> uint32_t {
+            const int64_t ss = tile * kBM + row;
+            return ss < N_c ? __ldg(reinterpret_cast<const uint32_t*>(k_scales + (b * N_c + ss) * 4)) : 0u;
         };
-        // tiles of this group: the valid tiles (tile * kBM < avail) with n_it % 2 == e
-        int64_t next_it[kSkAhead + 1];
-        uint32_t skq[kSkAhead];
-        auto advance = [&](int64_t from, int64_t& cnt) -> int64_t {   // next tile of group e
-            for (int64_t i = from; i < it1; ++i) {
-                const int64_t gg = i / tiles_per, tt = i - gg * tiles_per;
-                if (tt * kBM >= avail(q_pos, gg, m, N_c)) continue;
-                const int64_t c = cnt++;
-                if ((c & 1) == e) return i;
-            }
-            return it1;
-        };
-        int64_t cnt = 0;
-        next_it[0] = advance(it0, cnt);
-#pragma unroll
-        for (int i = 1; i <= kSkAhead; ++i) next_it[i] = advance(next_it[i - 1] + 1, cnt);
-#pragma unroll
-        for (int i = 0; i < kSkAhead; ++i) skq[i] = load_sk(next_it[i]);
-        while (next_it[0] < it1) {
-            const int64_t it = next_it[0];
-            const uint32_t skw = skq[0];
-#pragma unroll
-            for (int i = 0; i < kSkAhead; ++i) next_it[i] = next_it[i + 1];
-            next_it[kSkAhead] = advance(next_it[kSkAhead - 1] + 1, cnt);
-#pragma unroll
-            for (int i = 0; i + 1 < kSkAhead; ++i) skq[i] = skq[i + 1];
-            skq[kSkAhead - 1] = load_sk(next_it[kSkAhead - 1]);
-            const int64_t g = it / tiles_per, tile = it - g * tiles_per;
+        int64_t pf_id[2] = {-1, -1};
+        uint32_t pf_val[2] = {0u, 0u};
+        int64_t nv = 0;   // valid tiles of the sequence so far (both groups)
+        TileIt ti(it0, (int)tiles_per, (int)Q);
+        for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
+            const int64_t g = ti.g, tile = ti.tile;
             const int64_t n = avail(q_pos, g, m, N_c);
+            if (tile * kBM >= n) continue;
+            if (((nv++) & 1) != e) continue;
+            const uint32_t skw = (pf_id[0] == it) ? pf_val[0] : load_sk(ti.b, tile);
+            pf_id[0] = pf_id[1];
+            pf_val[0] = pf_val[1];
+            pf_id[1] = -1;
+            if (it + 4 < it1) {
+                TileIt t4 = ti;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) t4.next((int)tiles_per, (int)Q);
+                pf_id[1] = it + 4;
+                pf_val[1] = load_sk(t4.b, t4.tile);
+            }
             const float4* wg4 = reinterpret_cast<const float4*>(w + g * kHeads);   // L1-resident
             const int64_t s = tile * kBM + row;
             float sk[4];
@@ -290,14 +280,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             float acc = 0.f;
 #pragma unroll
-            for (int h0 = 0; h0 < kHeads; h0 += 16) {
-                uint32_t ev[4][16];
+            for (int h0 = 0; h0 < kHeads; h0 += 8) {
+                uint32_t ev[4][8];
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk)
-                    tmem_ld16(tmem_addr(tmem, quarter * 32, e * 256 + blk * 64 + h0), ev[blk]);
+                    tmem_ld8(tmem_addr(tmem, quarter * 32, e * 256 + blk * 64 + h0), ev[blk]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4) {
+                for (int j4 = 0; j4 < 2; ++j4) {
                     const float4 w4 = __ldg(wg4 + h0 / 4 + j4);
                     const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll

@@ -169,6 +169,29 @@ __device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
+// (group, tile, request) of a linear tile index it = g * tiles_per + tile, with
+// g = b * Q + q, advanced by one tile without integer division.
+struct TileIt {
+    int64_t g, b;
+    int tile, q;
+    __device__ __forceinline__ TileIt(int64_t it, int tiles_per, int Q) {
+        g = it / tiles_per;
+        tile = (int)(it - g * tiles_per);
+        b = g / Q;
+        q = (int)(g - b * Q);
+    }
+    __device__ __forceinline__ void next(int tiles_per, int Q) {
+        if (++tile == tiles_per) {
+            tile = 0;
+            ++g;
+            if (++q == Q) {
+                q = 0;
+                ++b;
+            }
+        }
+    }
+};
+
 // ------------------------------------------------------------ clusters / DSMEM
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -244,6 +267,13 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  : "memory");
 }
 
+// 32 lanes x 32 bits, 8 consecutive columns (thread i: lane base + i, register j: column
+// base + j).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
 // 32 lanes x 32 bits, 16 consecutive columns: thread i of the warp gets lane
 // (base lane + i), registers j = column (base column + j).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
