@@ -11,7 +11,7 @@
 // Tensor-core path (H = 64, D = 576, d_v = 512; bf16 rows or FP8 rows), 448 threads:
 //  * one CTA per (query, split of its row list); the row list is the window rows
 //    (padded to whole chunks of 64) followed by the selected (CSA) or available (HCA)
-//    compressed rows; the splits of a query form one thread-block cluster;
+//    compressed rows;
 //  * warp 12 loads the 64 query heads once (TMA, 128-byte swizzle) and issues
 //    tcgen05.mma with the query heads as M = 64:
 //      S [64 heads x 64 rows] = Q [64 x 576] . K_chunk^T        (K-major x K-major)
@@ -33,8 +33,7 @@
 //    own, rescale O in TMEM only when a head's running max grows by more than 2^8
 //    in weight, and write O / l out through shared memory (coalesced);
 //  * with several splits each CTA writes its unnormalised O and (m, l) to the
-//    workspace; after a cluster barrier CTA r merges heads r, r+splits, ... in split
-//    order.
+//    workspace, and attend_combine_kernel merges them in split order.
 // F32 path (C1-sized problems): CUDA cores, fp32 online softmax.
 #include <utility>
 
@@ -52,11 +51,10 @@ constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
 constexpr int kAtThreads = 448;   // 4 softmax, 8 producers, 1 Q.K^T issuer, 1 P.V issuer
 constexpr int kWarpQK = 12, kWarpPV = 13;
 constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kBlk;   // + the low part of P
-constexpr int kMaxSplits = 16;                // splits of one query form one cluster
+constexpr int kMaxSplits = 16;                // row-list splits per query (merged by attend_combine_kernel)
 constexpr int kOPitchF32 = kDv * 4 + 16;      // staged O rows (padded)
 constexpr int kOPitchBF16 = kDv * 2 + 16;
 static_assert(kH * kOPitchF32 <= 2 * kStageBytes, "staged O fits in the stages");
-static_assert((32 * kMaxSplits + 32) * 4 + 32 * kMaxSplits * 8 <= kBlk, "combine tables fit in the P_lo block");
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
@@ -147,14 +145,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* q_s = smem;
     uint8_t* stage_s = smem + kQBytes;
-    uint8_t* plo_s = stage_s + 2 * kStageBytes;   // low bf16 part of P (one block); after the
-                                                  // main loop, the combine's small tables
-    float* fac_s = reinterpret_cast<float*>(plo_s);             // [32][kMaxSplits]
-    float* inv_s = fac_s + 32 * kMaxSplits;                     // [32]
+    uint8_t* plo_s = stage_s + 2 * kStageBytes;   // low bf16 part of P (one block)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g = blockIdx.x / splits;
-    const int sp = blockIdx.x - (int)(g * splits);   // == rank in the query's cluster
+    const int sp = blockIdx.x - (int)(g * splits);
     const int64_t b = g / a.Q;
     constexpr int row_bytes = FP8 ? 656 : kD * 2;
 
@@ -507,7 +502,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             mbar_arrive(&bars.pfull[st]);
         }
         // ---- epilogue: O (normalised when this is the only split; else the partial O and
-        // (m, l) for the cluster combine) staged through shared memory, coalesced global
+        // (m, l) for the split combine) staged through shared memory, coalesced global
         // writes.  Lane l of warp q holds the O row of head 16q + (l & 15), dims 0-255
         // (lanes 0-15) or 256-511 (lanes 16-31).
         if (nch > 0) mbar_wait(&bars.odone, 0, status, 322);
@@ -571,89 +566,70 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
 
     tc_fence_before();
-    if (splits > 1) {
-        // ---- cluster combine: the splits of query g are the CTAs of one cluster.  Once
-        // every split's partial is in global memory (L2), CTA r merges heads r, r+splits, ...
-        // in split order.
-        __threadfence();
-        cluster_sync_all();
-        const uint32_t rank = cluster_ctarank();
-        const int nh = (kH - (int)rank + splits - 1) / splits;
-        const float* mlq = part_ml + g * splits * kH * 2;
-        const float* oq = part_o + g * splits * kH * kDv;
-        // (m, l) of every (head of this CTA, split): one load each, all in flight together
-        float2* mls = reinterpret_cast<float2*>(inv_s + 32);   // [32][kMaxSplits]
-        for (int t = threadIdx.x; t < nh * splits; t += blockDim.x) {
-            const int j = t / splits, s = t - j * splits;
-            mls[j * kMaxSplits + s] = __ldcg(reinterpret_cast<const float2*>(mlq) + s * kH + (int)rank + splits * j);
-        }
-        __syncthreads();
-        for (int j = threadIdx.x; j < nh; j += blockDim.x) {
-            const int h = (int)rank + splits * j;
-            float M = -INFINITY;
-            for (int s = 0; s < splits; ++s) M = fmaxf(M, mls[j * kMaxSplits + s].x);
-            float L = 0.f;
-            for (int s = 0; s < splits; ++s) {
-                const float2 ml = mls[j * kMaxSplits + s];
-                const float e = (ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
-                fac_s[j * kMaxSplits + s] = e;
-                L += ml.y * e;
-            }
-            inv_s[j] = L > 0.f ? 1.f / L : 0.f;
-            if (a.lse != nullptr) a.lse[g * kH + h] = L > 0.f ? (M + log2f(L)) / kLog2e : -INFINITY;
-        }
-        __syncthreads();
-        // O rows: a thread merges kItems (head, 4-dim) items at a time, their loads for one
-        // split in flight together
-        constexpr int kItems = 4;
-        const int n_items = nh * (kDv / 4);
-        for (int i0 = threadIdx.x; i0 < n_items; i0 += kItems * blockDim.x) {
-            float4 acc[kItems];
-#pragma unroll
-            for (int u = 0; u < kItems; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s = 0; s < splits; ++s) {
-                float4 v[kItems];
-#pragma unroll
-                for (int u = 0; u < kItems; ++u) {
-                    const int item = i0 + u * blockDim.x;
-                    const int j = item / (kDv / 4), d4 = item - j * (kDv / 4);
-                    v[u] = item < n_items
-                               ? __ldcg(reinterpret_cast<const float4*>(oq + (s * kH + (int)rank + splits * j) * kDv) + d4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int u = 0; u < kItems; ++u) {
-                    const int item = i0 + u * blockDim.x;
-                    const float e = item < n_items ? fac_s[(item / (kDv / 4)) * kMaxSplits + s] : 0.f;
-                    acc[u].x += v[u].x * e;
-                    acc[u].y += v[u].y * e;
-                    acc[u].z += v[u].z * e;
-                    acc[u].w += v[u].w * e;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kItems; ++u) {
-                const int item = i0 + u * blockDim.x;
-                if (item >= n_items) break;
-                const int j = item / (kDv / 4), d4 = item - j * (kDv / 4);
-                const int h = (int)rank + splits * j;
-                const float iv = inv_s[j];
-                const int64_t o = (g * kH + h) * kDv + d4 * 4;
-                if (a.out_dtype == LCS_F32) {
-                    *reinterpret_cast<float4*>(static_cast<float*>(a.out) + o) =
-                        make_float4(acc[u].x * iv, acc[u].y * iv, acc[u].z * iv, acc[u].w * iv);
-                } else {
-                    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + o) = make_uint2(
-                        pack_bf16x2(acc[u].x * iv, acc[u].y * iv), pack_bf16x2(acc[u].z * iv, acc[u].w * iv));
-                }
-            }
-        }
-    } else {
-        __syncthreads();
-    }
+    __syncthreads();
+#if defined(__CUDA_ARCH__)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the split combine
+#endif
     if (warp == kWarpQK) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// Merges the split partials of one (query, head) per CTA: 128 threads, one float4 of the
+// 512 output dims each.  The split weights exp2(m_s - M) and 1/L are formed once; every
+// split's float4 is loaded before any is used; the sum runs in split order.
+__global__ void __launch_bounds__(128) attend_combine_kernel(const float* __restrict__ part_o,
+                                                             const float* __restrict__ part_ml, int splits,
+                                                             void* __restrict__ out, int out_dtype,
+                                                             float* __restrict__ lse) {
+    __shared__ float fac[kMaxSplits];
+    __shared__ float inv_l;
+    const int64_t gh = blockIdx.x;   // query * 64 + head
+    const int64_t g = gh / kH;
+    const int h = (int)(gh - g * kH);
+    const int t = threadIdx.x;
+#if defined(__CUDA_ARCH__)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+    if (t < 32) {
+        float2 ml = make_float2(-INFINITY, 0.f);
+        if (t < splits) ml = __ldcg(reinterpret_cast<const float2*>(part_ml) + (g * splits + t) * kH + h);
+        float M = ml.x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float e = (t < splits && ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
+        if (t < splits) fac[t] = e;
+        // L summed in split order by lane 0
+        float L = 0.f;
+        for (int s = 0; s < splits; ++s) L += __shfl_sync(0xffffffffu, ml.y * e, s);
+        if (t == 0) {
+            inv_l = L > 0.f ? 1.f / L : 0.f;
+            if (lse != nullptr) lse[gh] = L > 0.f ? (M + log2f(L)) / kLog2e : -INFINITY;
+        }
+    }
+    __syncthreads();
+    const float4* src = reinterpret_cast<const float4*>(part_o) + (g * splits * kH + h) * (kDv / 4) + t;
+    float4 v[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s)
+        if (s < splits) v[s] = __ldcg(src + (int64_t)s * kH * (kDv / 4));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s)
+        if (s < splits) {
+            const float e = fac[s];
+            acc.x += v[s].x * e;
+            acc.y += v[s].y * e;
+            acc.z += v[s].z * e;
+            acc.w += v[s].w * e;
+        }
+    const float iv = inv_l;
+    if (out_dtype == LCS_F32) {
+        reinterpret_cast<float4*>(out)[gh * (kDv / 4) + t] = make_float4(acc.x * iv, acc.y * iv, acc.z * iv, acc.w * iv);
+    } else {
+        reinterpret_cast<uint2*>(out)[gh * (kDv / 4) + t] =
+            make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv), pack_bf16x2(acc.z * iv, acc.w * iv));
     }
 }
 
@@ -752,55 +728,18 @@ int64_t max_chunks(const AttendArgs& a) {
     return (nw + kChunk - 1) / kChunk + ((a.idx != nullptr ? a.k : a.N_c) + kChunk - 1) / kChunk;
 }
 
-const void* tc_kernel(const AttendArgs& a) {
-    return (a.kv_dtype == LCS_KV_FP8) ? reinterpret_cast<const void*>(attend_tc_kernel<true>)
-                                      : reinterpret_cast<const void*>(attend_tc_kernel<false>);
-}
-
-// How many clusters of `s` CTAs (one per SM: this kernel's shared memory) the device
-// keeps resident at once; cached per kernel and size.  Sizes above 8 are non-portable.
-int resident_clusters(const void* kern, int s) {
-    static std::mutex mu;
-    static int cache[2][kMaxSplits + 1];
-    const int which = (kern == reinterpret_cast<const void*>(attend_tc_kernel<true>));
-    std::lock_guard<std::mutex> lock(mu);
-    if (cache[which][s] == 0) {
-        int n = 0;
-        if (set_smem_once(kern, kAtSmem) == cudaSuccess &&
-            (s <= 8 || cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3((unsigned)s);
-            cfg.blockDim = dim3(kAtThreads);
-            cfg.dynamicSmemBytes = kAtSmem;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = (unsigned)s;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
-        }
-        cudaGetLastError();
-        cache[which][s] = n > 0 ? n : -1;
-    }
-    return cache[which][s];
-}
-
-// Splits per query: each query's splits form one cluster and every CTA of the launch is
-// resident at once (queries x splits <= SMs).  Picks the size that minimises the chunks
-// per CTA plus a fixed per-CTA cost of about two chunks (prologue, pipeline fill, epilogue
-// and combine), keeping at least two chunks per split.
+// Splits per query: every CTA of the launch resident at once (queries x splits <= SMs, one
+// CTA per SM), at least two chunks per split; picks the count that minimises the chunks per
+// CTA plus a fixed per-CTA cost of about two chunks (prologue, pipeline fill, epilogue) and,
+// with splits, one more for the combine.
 int choose_splits(const AttendArgs& a) {
     const int64_t queries = a.B * a.Q;
     const int64_t chunks = max_chunks(a);
-    const void* kern = tc_kernel(a);
     int best = 1;
     double best_cost = (double)chunks + 2.0;
     for (int s = 2; s <= kMaxSplits; ++s) {
         if ((chunks + s - 1) / s < 2 || queries * s > num_sms()) break;
-        if (resident_clusters(kern, s) < queries) continue;
-        const double cost = (double)((chunks + s - 1) / s) + 2.0;
+        const double cost = (double)((chunks + s - 1) / s) + 3.0;
         if (cost < best_cost) {
             best = s;
             best_cost = cost;
@@ -862,26 +801,11 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
         part_o = static_cast<float*>(scratch);
         part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256(queries * splits * kH * kDv * 4));
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(queries * splits));
-    cfg.blockDim = dim3(kAtThreads);
-    cfg.dynamicSmemBytes = kAtSmem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    int na = 0;
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = (unsigned)splits;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    ++na;
-    if (pdl) {
-        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, kern, mq, mc, mw, a, splits, part_o, part_ml, status);
+    e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, mc, mw, a, splits,
+                 part_o, part_ml, status);
+    if (e != cudaSuccess || splits == 1) return e;
+    return launch_k(attend_combine_kernel, dim3((unsigned)(queries * kH)), dim3(128), 0, s, true, part_o, part_ml,
+                    splits, a.out, a.out_dtype, a.lse);
 }
 
 }  // namespace lcs
