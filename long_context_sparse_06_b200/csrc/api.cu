@@ -158,6 +158,23 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, 
     return true;
 }
 
+// 3-D map over [outer2][outer1][inner] elements (rows of inner elements, row_stride bytes
+// apart; planes plane_stride bytes apart), box {box_inner, box_rows, 1}, no swizzle.
+// Out-of-range rows of a plane read as zeros.  Not cached (used by long-running calls).
+bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer1,
+                    uint64_t outer2, uint64_t row_stride_bytes, uint64_t plane_stride_bytes, uint32_t box_inner,
+                    uint32_t box_rows) {
+    EncodeTiledFn fn = get_encoder();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {inner, outer1, outer2};
+    cuuint64_t strides[2] = {row_stride_bytes, plane_stride_bytes};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace lcs
 
 using namespace lcs;

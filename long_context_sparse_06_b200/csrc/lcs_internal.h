@@ -97,5 +97,8 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer1,
+                    uint64_t outer2, uint64_t row_stride_bytes, uint64_t plane_stride_bytes, uint32_t box_inner,
+                    uint32_t box_rows);
 
 }  // namespace lcs

@@ -69,12 +69,14 @@ def test_rope(L, orc, dtype):
 
 
 # ------------------------------------------------------------------ compress
-@pytest.mark.parametrize("case", ["c1_f32", "csa_bf16_tail", "hca_bf16", "m1_identity"])
+@pytest.mark.parametrize("case", ["c1_f32", "csa_bf16_tail", "csa_bf16_notail", "hca_bf16", "m1_identity"])
 def test_compress(L, orc, case):
     if case == "c1_f32":
         B, T, d, m, ov, dr, dt, pos0 = 2, 1024, 64, 4, 2, 16, torch.float32, 0
     elif case == "csa_bf16_tail":
         B, T, d, m, ov, dr, dt, pos0 = 2, 260, 576, 4, 2, 64, torch.bfloat16, 131072
+    elif case == "csa_bf16_notail":   # 3 requests: the first window of each starts before its sequence
+        B, T, d, m, ov, dr, dt, pos0 = 3, 200, 128, 4, 2, 0, torch.bfloat16, 0
     elif case == "hca_bf16":
         B, T, d, m, ov, dr, dt, pos0 = 2, 128 * 5, 576, 128, 0, 64, torch.bfloat16, 0
     else:
