@@ -131,7 +131,8 @@ LCS_API int hca_compress(const void* x, int x_dtype, int64_t B, int64_t T, int d
  *   kI  [B, N_c, d_I]     see qI; LCS_FP4 uses the two-plane layout over B*N_c vectors
  *   q_pos [B, Q] int64 or NULL (then Q must be 1)
  *   idx [B, Q, k] int32 (out)
- *   scores [B, Q, N_c] score_dtype, optional output (NULL: kept in the workspace)
+ *   scores [B, Q, N_c] score_dtype, optional output (NULL: kept in the workspace);
+ *                         entries s >= n_avail are unspecified
  * score_dtype: LCS_F32 (kI F32 or BF16) or LCS_BF16 (kI FP4).  d_I % 32 == 0,
  * H_I <= 128 (LCS_F32 path) or H_I == 64 (tensor-core paths).
  */

@@ -63,51 +63,78 @@ __global__ void index_f32_kernel(const float* __restrict__ qI, const float* __re
 }
 
 // ------------------------------------------------------------- bf16 tcgen05 path
+// QB queries of one request share a group: their 64 x QB heads are the MMA's N, so each
+// key tile is read once per QB queries (decode: QB = 1; prefill: QB = 4, N = 256).
 constexpr int kBM = 128;        // keys per tile (MMA M)
-constexpr int kHeads = 64;      // index heads (MMA N)
+constexpr int kHeads = 64;      // index heads per query
 constexpr int kDI = 128;        // index dim (MMA K)
-constexpr int kStages = 4;
-constexpr int kAcc = 4;
 constexpr int kATile = kBM * kDI * 2;        // 32 KB
-constexpr int kBTile = kHeads * kDI * 2;     // 16 KB
-constexpr int kTmemCols = kAcc * kHeads;     // 256
 constexpr int kIxThreads = 192;
-constexpr size_t kIxSmem = 1024 + kStages * kATile + 2 * kBTile;
+template <int QB>
+struct IxCfg {
+    static constexpr int kN = kHeads * QB;                 // MMA N
+    static constexpr int kStages = QB == 1 ? 4 : 3;
+    static constexpr int kAcc = QB == 1 ? 4 : 2;
+    static constexpr int kBTile = kN * kDI * 2;            // 16 KB x QB
+    static constexpr int kTmemCols = kAcc * kN;            // 256 or 512
+    static constexpr size_t kSmem = 1024 + kStages * kATile + 2 * kBTile;
+};
 
+template <int QB>
 struct IxBars {
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[IxCfg<QB>::kStages], empty[IxCfg<QB>::kStages];
     uint64_t bfull[2], bempty[2];
-    uint64_t afull[kAcc], aempty[kAcc];
+    uint64_t afull[IxCfg<QB>::kAcc], aempty[IxCfg<QB>::kAcc];
     uint32_t tmem_base;
 };
 
+// Entries of group gb (request b, queries QB*qb ...) available to its last query.
+template <int QB>
+__device__ __forceinline__ int64_t group_avail(const int64_t* q_pos, int64_t b, int64_t qb, int64_t Q, int m,
+                                               int64_t N_c) {
+    if (q_pos == nullptr) return N_c;
+    int64_t n = 0;
+#pragma unroll
+    for (int qi = 0; qi < QB; ++qi) {
+        const int64_t q = qb * QB + qi;
+        if (q < Q) {
+            const int64_t a = avail(q_pos, b * Q + q, m, N_c);
+            n = a > n ? a : n;
+        }
+    }
+    return n;
+}
+
+template <int QB>
 __global__ void __launch_bounds__(kIxThreads, 1)
     index_bf16_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                          const float* __restrict__ w, int64_t Q, int64_t N_c, const int64_t* __restrict__ q_pos,
-                         int m, int64_t groups, float* __restrict__ scores, int* status) {
+                         int m, int64_t n_groups, float* __restrict__ scores, int* status) {
+    using C = IxCfg<QB>;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ IxBars bars;
+    __shared__ IxBars<QB> bars;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* a_tiles = smem;
-    uint8_t* b_tiles = smem + kStages * kATile;
+    uint8_t* b_tiles = smem + C::kStages * kATile;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nqb = (Q + QB - 1) / QB;   // groups per request
     const int64_t tiles_per = (N_c + kBM - 1) / kBM;
-    const int64_t total = groups * tiles_per;
+    const int64_t total = n_groups * tiles_per;
     const int64_t per = (total + gridDim.x - 1) / gridDim.x;
     const int64_t it0 = (int64_t)blockIdx.x * per;
     const int64_t it1 = (it0 + per < total) ? it0 + per : total;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) { mbar_init(&bars.full[i], 1); mbar_init(&bars.empty[i], 1); }
+        for (int i = 0; i < C::kStages; ++i) { mbar_init(&bars.full[i], 1); mbar_init(&bars.empty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&bars.bfull[i], 1); mbar_init(&bars.bempty[i], 1); }
-        for (int i = 0; i < kAcc; ++i) { mbar_init(&bars.afull[i], 1); mbar_init(&bars.aempty[i], 4); }
+        for (int i = 0; i < C::kAcc; ++i) { mbar_init(&bars.afull[i], 1); mbar_init(&bars.aempty[i], 4); }
         fence_barrier_init();
         prefetch_tmap(&map_k);
         prefetch_tmap(&map_q);
     }
     if (warp == 1) {
-        tmem_alloc(&bars.tmem_base, kTmemCols);
+        tmem_alloc(&bars.tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -124,41 +151,40 @@ __global__ void __launch_bounds__(kIxThreads, 1)
         if (lane == 0) {
             // ---------------- TMA producer
             int64_t prev_g = -1, gseq = -1, n_it = 0;
-            TileIt ti(it0, (int)tiles_per, (int)Q);
-            for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
+            TileIt ti(it0, (int)tiles_per, (int)nqb);
+            for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)nqb)) {
                 const int64_t g = ti.g, tile = ti.tile;
-                if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
+                if (tile * kBM >= group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c)) continue;
                 if (g != prev_g) {
                     ++gseq;
                     const int slot = (int)(gseq & 1);
                     if (!mbar_wait(&bars.bempty[slot], (uint32_t)(((gseq >> 1) & 1) ^ 1), status, 101)) break;
-                    mbar_arrive_expect_tx(&bars.bfull[slot], kBTile);
+                    mbar_arrive_expect_tx(&bars.bfull[slot], C::kBTile);
                     for (int kb = 0; kb < 2; ++kb)
-                        tma_load_2d(b_tiles + slot * kBTile + kb * (kBTile / 2), &map_q, &bars.bfull[slot], kb * 64,
-                                    (int)(g * kHeads));
+                        tma_load_2d(b_tiles + slot * C::kBTile + kb * (C::kBTile / 2), &map_q, &bars.bfull[slot],
+                                    kb * 64, (int)((ti.b * Q + ti.q * QB) * kHeads));
                     prev_g = g;
                 }
-                const int st = (int)(n_it % kStages);
-                if (!mbar_wait(&bars.empty[st], (uint32_t)(((n_it / kStages) & 1) ^ 1), status, 102)) break;
+                const int st = (int)(n_it % C::kStages);
+                if (!mbar_wait(&bars.empty[st], (uint32_t)(((n_it / C::kStages) & 1) ^ 1), status, 102)) break;
                 mbar_arrive_expect_tx(&bars.full[st], kATile);
-                const int64_t b = ti.b;
                 for (int kb = 0; kb < 2; ++kb)
                     tma_load_2d(a_tiles + st * kATile + kb * (kATile / 2), &map_k, &bars.full[st], kb * 64,
-                                (int)(b * N_c + tile * kBM));
+                                (int)(ti.b * N_c + tile * kBM));
                 ++n_it;
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
-            constexpr uint32_t idesc = idesc_bf16(kBM, kHeads, false, false);
+            constexpr uint32_t idesc = idesc_bf16(kBM, C::kN, false, false);
             int64_t prev_g = -1, gseq = -1, n_it = 0;
             int slot = 0;
             bool ok = true;
-            TileIt ti(it0, (int)tiles_per, (int)Q);
-            for (int64_t it = it0; it < it1 && ok; ++it, ti.next((int)tiles_per, (int)Q)) {
+            TileIt ti(it0, (int)tiles_per, (int)nqb);
+            for (int64_t it = it0; it < it1 && ok; ++it, ti.next((int)tiles_per, (int)nqb)) {
                 const int64_t g = ti.g, tile = ti.tile;
-                if (tile * kBM >= avail(q_pos, g, m, N_c)) continue;
+                if (tile * kBM >= group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c)) continue;
                 if (g != prev_g) {
                     if (prev_g >= 0) mma_commit(&bars.bempty[slot]);   // previous group's heads are free
                     ++gseq;
@@ -166,20 +192,20 @@ __global__ void __launch_bounds__(kIxThreads, 1)
                     if (!mbar_wait(&bars.bfull[slot], (uint32_t)((gseq >> 1) & 1), status, 103)) { ok = false; break; }
                     prev_g = g;
                 }
-                const int st = (int)(n_it % kStages);
-                const int ac = (int)(n_it % kAcc);
-                if (!mbar_wait(&bars.aempty[ac], (uint32_t)(((n_it / kAcc) & 1) ^ 1), status, 104)) { ok = false; break; }
-                if (!mbar_wait(&bars.full[st], (uint32_t)((n_it / kStages) & 1), status, 105)) { ok = false; break; }
+                const int st = (int)(n_it % C::kStages);
+                const int ac = (int)(n_it % C::kAcc);
+                if (!mbar_wait(&bars.aempty[ac], (uint32_t)(((n_it / C::kAcc) & 1) ^ 1), status, 104)) { ok = false; break; }
+                if (!mbar_wait(&bars.full[st], (uint32_t)((n_it / C::kStages) & 1), status, 105)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a_base = smem_u32(a_tiles + st * kATile);
-                const uint32_t b_base = smem_u32(b_tiles + slot * kBTile);
+                const uint32_t b_base = smem_u32(b_tiles + slot * C::kBTile);
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = sw128_desc(a_base + kb * (kATile / 2) + kk * 32, 16, 1024);
-                        const uint64_t bd = sw128_desc(b_base + kb * (kBTile / 2) + kk * 32, 16, 1024);
-                        mma_bf16_ss(tmem + ac * kHeads, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+                        const uint64_t bd = sw128_desc(b_base + kb * (C::kBTile / 2) + kk * 32, 16, 1024);
+                        mma_bf16_ss(tmem + ac * C::kN, ad, bd, idesc, (kb | kk) ? 1u : 0u);
                     }
                 mma_commit(&bars.empty[st]);
                 mma_commit(&bars.afull[ac]);
@@ -188,40 +214,47 @@ __global__ void __launch_bounds__(kIxThreads, 1)
             if (prev_g >= 0) mma_commit(&bars.bempty[slot]);
         }
     } else {
-        // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4
+        // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4, thread = key
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        int64_t prev_g = -1, n_it = 0;
-        float wr[kHeads];
-        TileIt ti(it0, (int)tiles_per, (int)Q);
-        for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)Q)) {
-            const int64_t g = ti.g, tile = ti.tile;
-            const int64_t n = avail(q_pos, g, m, N_c);
-            if (tile * kBM >= n) continue;
-            if (g != prev_g) {
-#pragma unroll
-                for (int h = 0; h < kHeads; ++h) wr[h] = __ldg(w + g * kHeads + h);
-                prev_g = g;
-            }
-            const int ac = (int)(n_it % kAcc);
-            if (!mbar_wait(&bars.afull[ac], (uint32_t)((n_it / kAcc) & 1), status, 106)) break;
+        int64_t n_it = 0;
+        TileIt ti(it0, (int)tiles_per, (int)nqb);
+        for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)nqb)) {
+            const int64_t tile = ti.tile;
+            if (tile * kBM >= group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c)) continue;
+            const int ac = (int)(n_it % C::kAcc);
+            if (!mbar_wait(&bars.afull[ac], (uint32_t)((n_it / C::kAcc) & 1), status, 106)) break;
             tc_fence_after();
-            uint32_t d[kHeads];
+            const int64_t s = tile * kBM + row;
+#pragma unroll 1
+            for (int qi = 0; qi < QB; ++qi) {
+                const int64_t q = ti.q * QB + qi;
+                uint32_t d[kHeads];
 #pragma unroll
-            for (int c = 0; c < kHeads / 16; ++c)
-                tmem_ld16(tmem_addr(tmem, quarter * 32, ac * kHeads + c * 16), *reinterpret_cast<uint32_t(*)[16]>(&d[c * 16]));
-            tmem_ld_wait();
+                for (int c = 0; c < kHeads / 16; ++c)
+                    tmem_ld16(tmem_addr(tmem, quarter * 32, ac * C::kN + qi * kHeads + c * 16),
+                              *reinterpret_cast<uint32_t(*)[16]>(&d[c * 16]));
+                tmem_ld_wait();
+                if (q >= Q) continue;
+                const int64_t gq = ti.b * Q + q;   // the query's row of qI, w, scores
+                const float4* w4 = reinterpret_cast<const float4*>(w + gq * kHeads);   // L1-resident
+                float acc = 0.f;
+#pragma unroll
+                for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+                    const float4 wv = __ldg(w4 + h4);
+                    const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float dot = __uint_as_float(d[4 * h4 + u]);
+                        acc = fmaf(ww[u], dot > 0.f ? dot : 0.f, acc);
+                    }
+                }
+                const int64_t n = avail(q_pos, gq, m, N_c);
+                if (s < N_c) scores[gq * N_c + s] = (s < n) ? acc : -INFINITY;
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.aempty[ac]);
-            float acc = 0.f;
-#pragma unroll
-            for (int h = 0; h < kHeads; ++h) {
-                const float dot = __uint_as_float(d[h]);
-                acc = fmaf(wr[h], dot > 0.f ? dot : 0.f, acc);
-            }
-            const int64_t s = tile * kBM + row;
-            if (s < N_c) scores[g * N_c + s] = (s < n) ? acc : -INFINITY;
             ++n_it;
         }
     }
@@ -230,7 +263,7 @@ __global__ void __launch_bounds__(kIxThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
@@ -259,16 +292,24 @@ cudaError_t launch_index_bf16_tc(const void* qI, const float* w, const void* kI,
     if (!encode_tmap_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kI, kDI, (uint64_t)(B * N_c), kDI * 2, 64, kBM,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    const bool batched = Q >= 4;   // prefill: four queries per group
+    const int qb = batched ? 4 : 1;
     if (!encode_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qI, kDI, (uint64_t)(groups * kHeads), kDI * 2, 64,
-                        kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
+                        (uint32_t)(kHeads * qb), CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    cudaError_t e =
-        set_smem_once(reinterpret_cast<const void*>(index_bf16_tc_kernel), kIxSmem);
-    if (e != cudaSuccess) return e;
-    const int64_t total = groups * ((N_c + kBM - 1) / kBM);
+    const int64_t n_groups = B * ((Q + qb - 1) / qb);
+    const int64_t total = n_groups * ((N_c + kBM - 1) / kBM);
     const int64_t grid = total < num_sms() ? total : num_sms();
-    return launch_k(index_bf16_tc_kernel, dim3((unsigned)grid), dim3(kIxThreads), kIxSmem, s, pdl, mk, mq, w, Q, N_c,
-                    q_pos, m, groups, scores, status);
+    if (batched) {
+        cudaError_t e = set_smem_once(reinterpret_cast<const void*>(index_bf16_tc_kernel<4>), IxCfg<4>::kSmem);
+        if (e != cudaSuccess) return e;
+        return launch_k(index_bf16_tc_kernel<4>, dim3((unsigned)grid), dim3(kIxThreads), IxCfg<4>::kSmem, s, pdl, mk,
+                        mq, w, Q, N_c, q_pos, m, n_groups, scores, status);
+    }
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(index_bf16_tc_kernel<1>), IxCfg<1>::kSmem);
+    if (e != cudaSuccess) return e;
+    return launch_k(index_bf16_tc_kernel<1>, dim3((unsigned)grid), dim3(kIxThreads), IxCfg<1>::kSmem, s, pdl, mk, mq,
+                    w, Q, N_c, q_pos, m, n_groups, scores, status);
 }
 
 }  // namespace lcs

@@ -195,21 +195,24 @@ def test_index_bf16_tensor_cores(L, orc):
     assert exact_rows >= B // 2
 
 
-def test_index_bf16_causal_prefill(L, orc):
-    B, Q, H, dI, Nc, k = 1, 40, 64, 128, 700, 64
-    qI = randn("g.ic.q", (B, Q, H, dI), dtype=torch.bfloat16)
-    w = randn("g.ic.w", (B, Q, H), std=1 / 8)
-    kI = randn("g.ic.k", (B, Nc, dI), dtype=torch.bfloat16)
-    q_pos = (torch.arange(Q, dtype=torch.int64) * 71 + 2).reshape(B, Q)
+@pytest.mark.parametrize("B,Q", [(1, 40), (2, 38)])   # 38: the last group of four queries is ragged
+def test_index_bf16_causal_prefill(L, orc, B, Q):
+    H, dI, Nc, k = 64, 128, 700, 64
+    qI = randn(f"g.ic.q{B}", (B, Q, H, dI), dtype=torch.bfloat16)
+    w = randn(f"g.ic.w{B}", (B, Q, H), std=1 / 8)
+    kI = randn(f"g.ic.k{B}", (B, Nc, dI), dtype=torch.bfloat16)
+    q_pos = (torch.arange(Q, dtype=torch.int64) * 71 + 2).reshape(1, Q).repeat(B, 1)
+    q_pos[B - 1] += 5
     idx, sc = L.csa_index_topk(qI.to(DEV), w.to(DEV), kI.to(DEV), k, q_pos=q_pos.to(DEV), m=4, want_scores=True)
     idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
-    for q in range(Q):
-        n = orc.n_avail(int(q_pos[0, q]), 4, Nc)
-        qd, kd, wd = qI[0, q].double().numpy(), kI[0, :n].double().numpy(), w[0, q].numpy()
-        ref = orc.index_scores_bf16(qd, wd, kd)
-        if n:
-            assert np.all(np.abs(sc[0, q, :n] - ref) <= _bf16_score_bound(qd, wd, kd))
-        np.testing.assert_array_equal(idx[0, q], orc.topk(sc[0, q, :n], k))
+    for b in range(B):
+        for q in range(Q):
+            n = orc.n_avail(int(q_pos[b, q]), 4, Nc)
+            qd, kd, wd = qI[b, q].double().numpy(), kI[b, :n].double().numpy(), w[b, q].numpy()
+            ref = orc.index_scores_bf16(qd, wd, kd)
+            if n:
+                assert np.all(np.abs(sc[b, q, :n] - ref) <= _bf16_score_bound(qd, wd, kd))
+            np.testing.assert_array_equal(idx[b, q], orc.topk(sc[b, q, :n], k))
 
 
 # ----------------------------------------------------------------- attention
