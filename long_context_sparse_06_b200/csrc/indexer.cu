@@ -152,9 +152,14 @@ __global__ void __launch_bounds__(kIxThreads, 1)
             // ---------------- TMA producer
             int64_t prev_g = -1, gseq = -1, n_it = 0;
             TileIt ti(it0, (int)tiles_per, (int)nqb);
+            int64_t av_g = -1, av_n = 0;
             for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)nqb)) {
                 const int64_t g = ti.g, tile = ti.tile;
-                if (tile * kBM >= group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c)) continue;
+                if (g != av_g) {   // availability of the group, formed once per group
+                    av_g = g;
+                    av_n = group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c);
+                }
+                if (tile * kBM >= av_n) continue;
                 if (g != prev_g) {
                     ++gseq;
                     const int slot = (int)(gseq & 1);
@@ -182,9 +187,14 @@ __global__ void __launch_bounds__(kIxThreads, 1)
             int slot = 0;
             bool ok = true;
             TileIt ti(it0, (int)tiles_per, (int)nqb);
+            int64_t av_g = -1, av_n = 0;
             for (int64_t it = it0; it < it1 && ok; ++it, ti.next((int)tiles_per, (int)nqb)) {
                 const int64_t g = ti.g, tile = ti.tile;
-                if (tile * kBM >= group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c)) continue;
+                if (g != av_g) {   // availability of the group, formed once per group
+                    av_g = g;
+                    av_n = group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c);
+                }
+                if (tile * kBM >= av_n) continue;
                 if (g != prev_g) {
                     if (prev_g >= 0) mma_commit(&bars.bempty[slot]);   // previous group's heads are free
                     ++gseq;
@@ -214,47 +224,67 @@ __global__ void __launch_bounds__(kIxThreads, 1)
             if (prev_g >= 0) mma_commit(&bars.bempty[slot]);
         }
     } else {
-        // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4, thread = key
+        // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4, thread = key.
+        // The QB queries' head chains run interleaved (each in its own fixed order h = 0..63),
+        // so that their fused multiply-adds hide one another's latency.
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        int64_t n_it = 0;
+        int64_t n_it = 0, av_g = -1, av_n = 0;
+        int64_t nq[QB];
+        const float4* wq[QB];
         TileIt ti(it0, (int)tiles_per, (int)nqb);
         for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)nqb)) {
             const int64_t tile = ti.tile;
-            if (tile * kBM >= group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c)) continue;
+            if (ti.g != av_g) {   // the group's queries: availability and head weights
+                av_g = ti.g;
+                av_n = 0;
+#pragma unroll
+                for (int qi = 0; qi < QB; ++qi) {
+                    const int64_t q = ti.q * QB + qi;
+                    const int64_t gq = ti.b * Q + (q < Q ? q : ti.q * QB);
+                    nq[qi] = q < Q ? avail(q_pos, gq, m, N_c) : -1;
+                    av_n = nq[qi] > av_n ? nq[qi] : av_n;
+                    wq[qi] = reinterpret_cast<const float4*>(w + gq * kHeads);   // L1-resident
+                }
+            }
+            if (tile * kBM >= av_n) continue;
             const int ac = (int)(n_it % C::kAcc);
             if (!mbar_wait(&bars.afull[ac], (uint32_t)((n_it / C::kAcc) & 1), status, 106)) break;
             tc_fence_after();
-            const int64_t s = tile * kBM + row;
+            float acc[QB];
+#pragma unroll
+            for (int qi = 0; qi < QB; ++qi) acc[qi] = 0.f;
 #pragma unroll 1
-            for (int qi = 0; qi < QB; ++qi) {
-                const int64_t q = ti.q * QB + qi;
-                uint32_t d[kHeads];
+            for (int h0 = 0; h0 < kHeads; h0 += 16) {
+                uint32_t d[QB][16];
 #pragma unroll
-                for (int c = 0; c < kHeads / 16; ++c)
-                    tmem_ld16(tmem_addr(tmem, quarter * 32, ac * C::kN + qi * kHeads + c * 16),
-                              *reinterpret_cast<uint32_t(*)[16]>(&d[c * 16]));
+                for (int qi = 0; qi < QB; ++qi)
+                    tmem_ld16(tmem_addr(tmem, quarter * 32, ac * C::kN + qi * kHeads + h0), d[qi]);
                 tmem_ld_wait();
-                if (q >= Q) continue;
-                const int64_t gq = ti.b * Q + q;   // the query's row of qI, w, scores
-                const float4* w4 = reinterpret_cast<const float4*>(w + gq * kHeads);   // L1-resident
-                float acc = 0.f;
 #pragma unroll
-                for (int h4 = 0; h4 < kHeads / 4; ++h4) {
-                    const float4 wv = __ldg(w4 + h4);
-                    const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    float4 wv[QB];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float dot = __uint_as_float(d[4 * h4 + u]);
-                        acc = fmaf(ww[u], dot > 0.f ? dot : 0.f, acc);
-                    }
+                    for (int qi = 0; qi < QB; ++qi) wv[qi] = __ldg(wq[qi] + h0 / 4 + j4);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+#pragma unroll
+                        for (int qi = 0; qi < QB; ++qi) {
+                            const float ww = u == 0 ? wv[qi].x : u == 1 ? wv[qi].y : u == 2 ? wv[qi].z : wv[qi].w;
+                            const float dot = __uint_as_float(d[qi][4 * j4 + u]);
+                            acc[qi] = fmaf(ww, dot > 0.f ? dot : 0.f, acc[qi]);
+                        }
                 }
-                const int64_t n = avail(q_pos, gq, m, N_c);
-                if (s < N_c) scores[gq * N_c + s] = (s < n) ? acc : -INFINITY;
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.aempty[ac]);
+            const int64_t s = tile * kBM + row;
+            if (s < N_c)
+#pragma unroll
+                for (int qi = 0; qi < QB; ++qi)
+                    if (nq[qi] >= 0)
+                        scores[(ti.b * Q + ti.q * QB + qi) * N_c + s] = (s < nq[qi]) ? acc[qi] : -INFINITY;
             ++n_it;
         }
     }
