@@ -311,27 +311,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // ---- selection length (CSA: the valid prefix of idx, as top-k emits it; HCA: n_avail).
     // An index >= N_c ends the prefix and is reported through the status word.
     if (a.idx != nullptr) {
-        if (warp == 0) {
-            int first_bad = a.k;
-            for (int base = 0; base < a.k; base += 256) {
-                int32_t v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i = base + 32 * j + lane;
-                    v[j] = (i < a.k) ? __ldg(sel + i) : 0;
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i = base + 32 * j + lane;
-                    if (i < a.k && (v[j] < 0 || v[j] >= a.N_c)) {
-                        if (v[j] >= a.N_c) set_status(status, LCS_ERR_DEVICE, 201);
-                        first_bad = min(first_bad, i);
-                    }
-                }
+        // every thread checks a few entries (one load round), then a block minimum
+        if (threadIdx.x == 0) bars.nsel = a.k;
+        __syncthreads();
+        int first_bad = a.k;
+        for (int i = threadIdx.x; i < a.k; i += kAtThreads) {
+            const int32_t v = __ldg(sel + i);
+            if (v < 0 || v >= a.N_c) {
+                if (v >= a.N_c) set_status(status, LCS_ERR_DEVICE, 201);
+                first_bad = min(first_bad, i);
             }
-            first_bad = __reduce_min_sync(0xffffffffu, first_bad);
-            if (lane == 0) bars.nsel = first_bad;
         }
+        first_bad = __reduce_min_sync(0xffffffffu, first_bad);
+        if (lane == 0 && first_bad < a.k) atomicMin(&bars.nsel, first_bad);
     } else if (threadIdx.x == 0) {
         bars.nsel = (int)comp_max;
     }
@@ -545,14 +537,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 }
             }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 softmax warps
-        const int row_bytes_out = f32 ? kDv * 4 : kDv * 2;
-        uint8_t* gout = final_out ? static_cast<uint8_t*>(a.out) + g * kH * row_bytes_out
-                                  : reinterpret_cast<uint8_t*>(part_o + (g * splits + sp) * kH * kDv);
-        for (int off = (int)threadIdx.x * 16; off < kH * row_bytes_out; off += 128 * 16) {
-            const int h = off / row_bytes_out, cb = off - h * row_bytes_out;
-            *reinterpret_cast<uint4*>(gout + off) = *reinterpret_cast<const uint4*>(ostage + h * row_pitch + cb);
-        }
         if (lane < 16) {
             if (final_out) {
                 if (a.lse != nullptr)
@@ -567,6 +551,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    {
+        // the staged O rows (normalised output, or this split's fp32 partial) go out with
+        // coalesced 16-byte stores from every thread of the CTA
+        const bool f32 = splits > 1 || a.out_dtype == LCS_F32;
+        const int row_pitch = f32 ? kOPitchF32 : kOPitchBF16;
+        const int row_bytes_out = f32 ? kDv * 4 : kDv * 2;
+        uint8_t* gout = splits == 1 ? static_cast<uint8_t*>(a.out) + g * kH * row_bytes_out
+                                    : reinterpret_cast<uint8_t*>(part_o + (g * splits + sp) * kH * kDv);
+        for (int off = (int)threadIdx.x * 16; off < kH * row_bytes_out; off += kAtThreads * 16) {
+            const int h = off / row_bytes_out, cb = off - h * row_bytes_out;
+            *reinterpret_cast<uint4*>(gout + off) = *reinterpret_cast<const uint4*>(stage_s + h * row_pitch + cb);
+        }
+    }
 #if defined(__CUDA_ARCH__)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the split combine
 #endif
