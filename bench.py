@@ -587,15 +587,44 @@ LAUNCHES_PER_STEP = {"csa_decode_bf16_128k": 4, "csa_decode_mixed_1m": 5, "hca_d
                      "csa_prefill_bf16_8k": 5, "compress_stream_1m": 3}
 
 
+# ------------------------------------------------------------- ranks (N > 1)
+# One process per GPU; requests are independent, so every rank runs its own replica of the
+# workload and the only cross-rank traffic is the timing: barriers around the timed region
+# and the maximum of the per-rank step times.
+def rank_env():
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world, device):
+    """The largest of the ranks' values (the job's step time is that of its slowest rank)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, units_per_rank_step, ms_step):
+    """Whole-job throughput: the units every rank processed per step over the step time."""
+    return world * units_per_rank_step / (ms_step / 1e3)
+
+
 # ------------------------------------------------------------------- GPU arm
 def run_gpu(args):
     import torch
     import torch.distributed as dist
     import long_context_sparse_06_b200 as lcs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
@@ -620,17 +649,6 @@ def run_gpu(args):
         print(json.dumps({"workload": wl.name, "stage": args.stage, "ms": e0.elapsed_time(e1) / args.steps}))
         return None
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     workspaces = [getattr(wl, a) for a in ("ws", "ws_i", "ws_a") if hasattr(wl, a)]
     for _ in range(args.warmup):
         wl.step(stream)
@@ -652,7 +670,7 @@ def run_gpu(args):
     # ---- timed region: K steps of the whole path (inputs larger than L2)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
-    barrier()
+    barrier(world)
     torch.cuda.synchronize()
     with sampler:
         e0.record(stream)
@@ -660,14 +678,14 @@ def run_gpu(args):
             graph.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-    barrier()
-    ms_step = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-    value = world * wl.units_per_step() / (ms_step / 1e3)
+    barrier(world)
+    ms_step = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    value = job_value(world, wl.units_per_step(), ms_step)
 
     # ---- stage times on the launching stream (library events between stages, or events
     # around separate calls); stages then run without programmatic overlap
     stage_ms = time_stages(wl, lcs, stream, args.steps, torch)
-    stage_ms = {k: max_over_ranks(v) for k, v in stage_ms.items()}
+    stage_ms = {k: max_over_ranks(v, world, dev) for k, v in stage_ms.items()}
 
     # ---- end to end through the public API: per-step inputs H2D from pinned host, result D2H
     ins, res_t = wl.e2e_io()
@@ -685,14 +703,14 @@ def run_gpu(args):
     for _ in range(max(3, args.warmup)):
         e2e_step()
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     e0.record(stream)
     for _ in range(args.steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
     for ws in workspaces:
         st = lcs.lcs_status(ws)
         if st != 0:
@@ -715,7 +733,7 @@ def run_gpu(args):
     else:
         dom_ms = (wl.dominant_ms(stream, args.steps, torch) if hasattr(wl, "dominant_ms")
                   else list(stage_ms.values())[wl.dominant_stage()])
-        dom_ms = max_over_ranks(dom_ms)
+        dom_ms = max_over_ranks(dom_ms, world, dev)
         achieved = wl.dominant_bytes() / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": wl.dominant, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "peak_source": f"{peak_kind} copy bandwidth",
@@ -742,7 +760,7 @@ def run_gpu(args):
                            parallelism=f"replicas x{world} (requests independent)"),
             "roofline": roof, "step_roofline": step_roof,
             "stage_ms": {k: round(v, 5) for k, v in stage_ms.items()},
-            "e2e": {"value": round(world * wl.units_per_step() / (e2e_ms / 1e3), 1), "unit": wl.unit,
+            "e2e": {"value": round(job_value(world, wl.units_per_step(), e2e_ms), 1), "unit": wl.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
                     "inputs": "per-step inputs H2D from pinned host, result D2H; caches resident"},
             "gpu_launches": args.steps * LAUNCHES_PER_STEP[wl.name],
@@ -825,8 +843,9 @@ def time_stages(wl, lcs, stream, steps, torch):
 
 # ------------------------------------------------------------- reference arm
 def run_reference(args):
-    """The oracle as the reference arm: each step is a bounded sample of the workload."""
-    rank = int(os.environ.get("RANK", "0"))
+    """The oracle as the reference arm: each step is a bounded sample of the workload.  Under
+    torchrun only rank 0 runs it; the other ranks return without work."""
+    rank = rank_env()[1]
     if rank != 0:
         return None
     import numpy as np
