@@ -68,8 +68,8 @@ KERNEL_FILES = {
                             "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
     "attend_tc_kernel": ["long_context_sparse_06_b200/csrc/attend.cu",
                          "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
-    "compress_kernel": ["long_context_sparse_06_b200/csrc/compress.cu",
-                        "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
+    "compress_tma_kernel": ["long_context_sparse_06_b200/csrc/compress.cu",
+                            "long_context_sparse_06_b200/csrc/lcs_common.cuh"],
 }
 
 
@@ -508,7 +508,7 @@ class CompressStream(Workload):
     unit = "tok/s"
     T = 1 << 20
     stage_names = ("csa_kv", "csa_index_keys", "hca_kv")
-    dominant = "compress_kernel"
+    dominant = "compress_tma_kernel"
 
     def config(self):
         return dict(workload=self.name, raw_tokens=self.T, kv_dim=D, index_dim=DI, csa_m=4, csa_overlap=2,
