@@ -382,6 +382,55 @@ class HcaDecode(Workload):
         return n, el, f"{n} of {self.B} requests, dense attention over {self.NC}+{TW} rows each; single thread"
 
 
+class HcaDecodeFp8(HcaDecode):
+    """HCA decode over FP8 rows (the 1M-context mixed-precision row format)."""
+    name = "hca_decode_fp8_1m"
+    row = 656
+
+    def config(self):
+        return dict(super().config(), workload=self.name,
+                    kv_format="fp8-e4m3 (pow2 scale per 128) + bf16 rope")
+
+    def build(self):
+        import torch
+        from long_context_sparse_06_b200 import synth
+        L, dev = self.lcs, self.dev
+        f32 = torch.float32
+        self.q = synth.normal_t(self.tag("q"), (self.B, H, D), dtype=torch.bfloat16, device=dev)
+        self.comp = L.lcs_quant_kv_fp8(synth.normal_t(self.tag("comp"), (self.B, self.NC, D), dtype=f32, device=dev))
+        self.win = L.lcs_quant_kv_fp8(synth.normal_t(self.tag("win"), (self.B, TW, D), dtype=f32, device=dev))
+        self.out = torch.empty((self.B, H, DV), dtype=torch.bfloat16, device=dev)
+        self.ws = L.workspace(L.lcs_workspace_size(L.OP_DECODE, self.B, 1, self.NC, TW, 0, H, DV), dev)
+
+    def step(self, stream):
+        L = self.lcs
+        L.decode_fused(L.MODE_HCA, self.q, self.comp, self.win, DV, SCALE, kv_dtype=L.KV_FP8, out=self.out,
+                       ws=self.ws, stream=stream)
+
+    def alg_bytes_per_step(self):
+        return self.B * ((self.NC + TW) * self.row + H * D * 2 + H * DV * 2)
+
+    def dominant_ms(self, stream, K, torch):
+        L = self.lcs
+        fn = lambda: L._call("hca_attend", L._ptr(self.q), L.BF16, L._ptr(self.comp), L._ptr(self.win), L.KV_FP8,
+                             self.B, 1, self.NC, TW, None, None, 128, TW, H, D, DV, SCALE, L._ptr(self.out), L.BF16,
+                             None, L._ptr(self.ws), self.ws.numel(), L._stream(stream))
+        return _time_launches(fn, stream, K, torch)
+
+    def cpu_sample(self, budget_s):
+        from oracle import oracle as orc
+        el, n = 0.0, 0
+        while n < self.B and el < budget_s:
+            q = self.q[n].double().cpu().numpy()
+            comp = orc.dequant_kv_fp8(self.comp[n].cpu().numpy())
+            win = orc.dequant_kv_fp8(self.win[n].cpu().numpy())
+            ts = time.perf_counter()
+            orc.hca_attend(q, comp, 128, win, 0, -1, TW, DV, SCALE)
+            el += time.perf_counter() - ts
+            n += 1
+        return n, el, f"{n} of {self.B} requests, dense attention over {self.NC}+{TW} FP8 rows each; single thread"
+
+
 class CsaPrefill(Workload):
     """Chunked prefill: 8192 new tokens after a 131072-token prefix."""
     name = "csa_prefill_bf16_8k"
@@ -582,8 +631,9 @@ class CompressStream(Workload):
                               f"scaled by that pass's share of the step's bytes; single thread"
 
 
-WORKLOADS = {c.name: c for c in (CsaDecode, HcaDecode, CsaDecodeMixed, CsaPrefill, CompressStream)}
+WORKLOADS = {c.name: c for c in (CsaDecode, HcaDecode, HcaDecodeFp8, CsaDecodeMixed, CsaPrefill, CompressStream)}
 LAUNCHES_PER_STEP = {"csa_decode_bf16_128k": 4, "csa_decode_mixed_1m": 5, "hca_decode_bf16_1m": 2,
+                     "hca_decode_fp8_1m": 2,
                      "csa_prefill_bf16_8k": 5, "compress_stream_1m": 3}
 
 

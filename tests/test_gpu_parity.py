@@ -302,6 +302,26 @@ def test_hca_attend_decode_tc(L, orc):
         assert_close_abs(lse[b, 0], l, 2e-2, f"hca lse b {b}")
 
 
+def test_hca_attend_decode_fp8(L, orc):
+    """HCA over FP8 rows (content E4M3 with a power-of-two scale per 128, RoPE dims bf16),
+    heavy-tailed values: the 1M-context row format applied to dense attention."""
+    from long_context_sparse_06_b200 import synth
+    B, H, D, dv, Nc, Tw = 3, 64, 576, 512, 1100, 128
+    scale = 1 / math.sqrt(576)
+    q = randn("g.h8.q", (B, 1, H, D), dtype=torch.bfloat16)
+    comp32 = synth.with_outliers("g.h8.c", synth.normal("g.h8.c", (B, Nc, D))).astype(np.float32)
+    win32 = synth.with_outliers("g.h8.w", synth.normal("g.h8.w", (B, Tw, D))).astype(np.float32)
+    comp_g = L.lcs_quant_kv_fp8(torch.from_numpy(comp32).to(DEV))
+    win_g = L.lcs_quant_kv_fp8(torch.from_numpy(win32).to(DEV))
+    out = both_outputs(lambda od: L.hca_attend(q.to(DEV), comp_g, win_g, dv, scale, kv_dtype=L.KV_FP8,
+                                               out_dtype=od)).cpu().numpy()
+    comp_d = orc.dequant_kv_fp8(orc.quant_kv_fp8(comp32))
+    win_d = orc.dequant_kv_fp8(orc.quant_kv_fp8(win32))
+    for b in range(B):
+        o, _ = orc.hca_attend(q[b, 0].double().numpy(), comp_d[b], 128, win_d[b], 0, -1, 128, dv, scale)
+        assert_close_rel_rms(out[b, 0], o, 2e-2, f"hca fp8 b {b}")
+
+
 @pytest.mark.parametrize("tail", [127, 50])
 def test_attend_prefill_tc_causal(L, orc, tail):
     """C4-shaped (smaller): queries at positions p0.., window from the chunk plus a prefix tail
