@@ -66,6 +66,7 @@ struct AtBars {
     uint64_t pfull[2];
     uint64_t ofull[2];   // P.V of chunk c done (per chunk parity)
     uint64_t odone;      // every P.V of this CTA done
+    uint64_t rawfull[2]; // FP8 chunk codes landed (TMA), before widening
     uint32_t tmem_base;
     int nsel;
 };
@@ -75,6 +76,45 @@ struct RowPlan {
     int64_t win_lo;      // first window row index in win[b]
     int64_t nwin;
 };
+
+// Named barrier of the `count` threads of one producer group.
+__device__ __forceinline__ void group_bar(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// AND of v over the `count` threads of one producer group (every thread reaches it once),
+// so that the group takes one decision after per-thread bounded waits.
+__device__ __forceinline__ bool group_all(int id, int count, bool v) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 q, %1, 0;\n\tbar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((int)v), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+// 16 E4M3 codes (a uint4, low byte first) times the power-of-two block scale s -> 16 bf16,
+// exact: code -> fp32 is exact, the product with a power of two is exact in fp32 and
+// representable in bf16, so the final rounding changes nothing.
+__device__ __forceinline__ void widen16(uint4 v, float s, uint32_t (&o)[8]) {
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        o[2 * q] = pack_bf16x2(e4m3_to_f32(w4[q] & 0xFF) * s, e4m3_to_f32((w4[q] >> 8) & 0xFF) * s);
+        o[2 * q + 1] = pack_bf16x2(e4m3_to_f32((w4[q] >> 16) & 0xFF) * s, e4m3_to_f32(w4[q] >> 24) * s);
+    }
+}
+
+// 16 codes of one row (a uint4) -> 16 bf16 written as the row's 16-byte chunks ch, ch+1
+// of a SW128 column block.
+__device__ __forceinline__ void widen_piece(uint8_t* blk, int r, int ch, uint4 v, float s) {
+    uint32_t o[8];
+    widen16(v, s, o);
+    *reinterpret_cast<uint4*>(blk + sw128_off(r, ch)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(blk + sw128_off(r, ch + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+}
 
 __device__ __forceinline__ RowPlan plan_rows(const AttendArgs& a, int64_t g, int nsel) {
     RowPlan p;
@@ -138,7 +178,8 @@ __device__ __forceinline__ int64_t hca_avail(const AttendArgs& a, int64_t g) {
 template <bool FP8>
 __global__ void __launch_bounds__(kAtThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_c,
-                     const __grid_constant__ CUtensorMap map_w, const AttendArgs a, int splits,
+                     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_cr,
+                     const __grid_constant__ CUtensorMap map_wr, const AttendArgs a, int splits,
                      float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ AtBars bars;
@@ -162,13 +203,16 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             mbar_init(&bars.sfull[i], 1);
             mbar_init(&bars.sempty[i], 128);
             mbar_init(&bars.ofull[i], 1);
+            mbar_init(&bars.rawfull[i], 1);
         }
         mbar_init(&bars.odone, 1);
         fence_barrier_init();
         prefetch_tmap(&map_q);
-        if constexpr (!FP8) {
-            prefetch_tmap(&map_c);
-            prefetch_tmap(&map_w);
+        prefetch_tmap(&map_c);
+        prefetch_tmap(&map_w);
+        if constexpr (FP8) {
+            prefetch_tmap(&map_cr);
+            prefetch_tmap(&map_wr);
         }
     }
     if (warp == kWarpQK) {
@@ -205,14 +249,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     };
 
     // ---- producers: warps 4-7 fill stage 0 (local chunks 0, 2, ...), warps 8-11 stage 1.
-    // Contiguous bf16 chunks (window rows; HCA's compressed rows) are one TMA tile load per
-    // 128-byte column block, issued by the group's first thread; selected rows (CSA) are
-    // gathered with 16-byte cp.async, warp pw of the group owning rows pw, pw+4, ..., pw+60
-    // (lane i < 16 resolves row pw+4i); FP8 rows are loaded, converted to bf16 (exact with
-    // the power-of-two block scale) and stored.  All write the SW128 layout both MMAs read.
+    // A whole chunk of consecutive rows (window rows; HCA's compressed rows) comes by TMA,
+    // issued by the group's first thread: bf16 rows as one tile load per 128-byte column
+    // block; FP8 rows as their codes, which the group then widens to bf16 in shared memory.
+    // Other chunks are gathered row by row, warp pw of the group owning rows pw, pw+4, ...,
+    // pw+60 (lane i < 16 resolves row pw+4i): bf16 rows with 16-byte cp.async, FP8 rows
+    // loaded, converted (exact with the power-of-two block scale) and stored.  The gathers
+    // write zeros for rows past the chunk's valid count, so a partial chunk never reads
+    // rows outside the query's row set (they may hold anything, NaN included).  All write
+    // the SW128 layout both MMAs read.
     const bool producer = warp >= 4 && warp < 12;
     const int pst = (warp - 4) >> 2, pw = (warp - 4) & 3;
-    auto contiguous = [&](int64_t gc) { return !FP8 && (gc < nwc || sel == nullptr); };
+    auto contiguous = [&](int64_t gc) { return (gc < nwc || sel == nullptr) && chunk_valid(gc) == kChunk; };
+    uint32_t raw_fills = 0;   // FP8 TMA fills of this group so far (rawfull parity)
     auto row_src = [&](int64_t gc, int rr) -> const uint8_t* {
         if (rr >= chunk_valid(gc)) return nullptr;
         if (gc < nwc)
@@ -228,16 +277,62 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     auto fill = [&](int64_t gc, const uint8_t* my_src) {
         uint8_t* dst = stage_s + pst * kStageBytes;
         if (contiguous(gc)) {
-            if (pw == 0 && lane == 0) {
-                mbar_arrive_expect_tx(&bars.kfull[pst], kStageBytes);
-                const bool w = gc < nwc;
-                const int row0 = w ? (int)(b * a.Tw + wp.win_lo + gc * kChunk) : (int)(b * a.N_c + (gc - nwc) * kChunk);
-                for (int blk = 0; blk < 9; ++blk)
-                    tma_load_2d(dst + blk * kBlk, w ? &map_w : &map_c, &bars.kfull[pst], blk * 64, row0);
+            const bool w = gc < nwc;
+            const int row0 = w ? (int)(b * a.Tw + wp.win_lo + gc * kChunk) : (int)(b * a.N_c + (gc - nwc) * kChunk);
+            if constexpr (!FP8) {
+                if (pw == 0 && lane == 0) {
+                    mbar_arrive_expect_tx(&bars.kfull[pst], kStageBytes);
+                    for (int blk = 0; blk < 9; ++blk)
+                        tma_load_2d(dst + blk * kBlk, w ? &map_w : &map_c, &bars.kfull[pst], blk * 64, row0);
+                } else {
+                    mbar_arrive(&bars.kfull[pst]);
+                }
+                return;
             } else {
+                // the codes of column block j (64 rows x 64 B) land in the upper half of
+                // block j, the RoPE dims (bf16, 128-byte swizzle) in block 8; thread tg then
+                // widens 16 codes of rows tg/4 and tg/4 + 32 per block (piece tg%4), reading
+                // block j+1's codes before the group barrier that lets block j+1 be written
+                const int tg = pw * 32 + lane;
+                if (tg == 0) {
+                    mbar_arrive_expect_tx(&bars.rawfull[pst], 8 * (kBlk / 2) + kBlk);
+                    for (int j = 0; j < 8; ++j)
+                        tma_load_2d(dst + j * kBlk + kBlk / 2, w ? &map_w : &map_c, &bars.rawfull[pst], j * 64, row0);
+                    tma_load_2d(dst + 8 * kBlk, w ? &map_wr : &map_cr, &bars.rawfull[pst], 512, row0);
+                }
+                const int r1 = tg >> 2, piece = tg & 3;
+                const uint8_t* scales = static_cast<const uint8_t*>(w ? a.win : a.comp) + (int64_t)row0 * 656 + 640;
+                const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + (int64_t)r1 * 656));
+                const float4 s2 = __ldg(reinterpret_cast<const float4*>(scales + (int64_t)(r1 + 32) * 656));
+                const bool landed =
+                    group_all(1 + pst, 128, mbar_wait(&bars.rawfull[pst], raw_fills & 1u, status, 311));
+                ++raw_fills;
+                if (landed) {
+                    const uint4* raw0 = reinterpret_cast<const uint4*>(dst + kBlk / 2);
+                    uint4 c1 = raw0[tg], c2 = raw0[tg + 128];
+                    group_bar(1 + pst, 128);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        uint4 n1 = c1, n2 = c2;
+                        if (j < 7) {
+                            const uint4* rawn = reinterpret_cast<const uint4*>(dst + (j + 1) * kBlk + kBlk / 2);
+                            n1 = rawn[tg];
+                            n2 = rawn[tg + 128];
+                        }
+                        const int sj = j >> 1;
+                        const float f1 = sj == 0 ? s1.x : sj == 1 ? s1.y : sj == 2 ? s1.z : s1.w;
+                        const float f2 = sj == 0 ? s2.x : sj == 1 ? s2.y : sj == 2 ? s2.z : s2.w;
+                        widen_piece(dst + j * kBlk, r1, 2 * piece, c1, f1);
+                        widen_piece(dst + j * kBlk, r1 + 32, 2 * piece, c2, f2);
+                        if (j < 7) group_bar(1 + pst, 128);
+                        c1 = n1;
+                        c2 = n2;
+                    }
+                }
+                fence_proxy_async_smem();
                 mbar_arrive(&bars.kfull[pst]);
+                return;
             }
-            return;
         }
         if constexpr (!FP8) {
 #pragma unroll 4
@@ -274,20 +369,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int rr = pw + 4 * (i0 + u);
-                    const uint32_t w4[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
-                    uint32_t o[8];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        o[2 * q] =
-                            pack_bf16x2(e4m3_to_f32(w4[q] & 0xFF) * sc[u], e4m3_to_f32((w4[q] >> 8) & 0xFF) * sc[u]);
-                        o[2 * q + 1] =
-                            pack_bf16x2(e4m3_to_f32((w4[q] >> 16) & 0xFF) * sc[u], e4m3_to_f32(w4[q] >> 24) * sc[u]);
-                    }
-                    const int ch = lane * 2;
-                    *reinterpret_cast<uint4*>(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<uint4*>(dst + ((ch + 1) >> 3) * kBlk + sw128_off(rr, (ch + 1) & 7)) =
-                        make_uint4(o[4], o[5], o[6], o[7]);
+                    // lane's 16 codes are the row's chunks 2*lane, 2*lane+1: block lane/4
+                    widen_piece(dst + (lane >> 2) * kBlk, rr, (lane & 3) * 2, cv[u], sc[u]);
                     if (lane < 8) *reinterpret_cast<uint4*>(dst + 8 * kBlk + sw128_off(rr, lane)) = rv[u];
                 }
             }
@@ -394,7 +477,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         for (int c = pst; c < nch; c += 2) {
             const uint8_t* my_src = nxt;
             const int u = c >> 1;
-            if (u >= 1 && !mbar_wait(&bars.kempty[pst], (uint32_t)((u - 1) & 1), status, 310)) break;
+            // the group leaves together (the FP8 widening syncs on group barriers)
+            if (u >= 1 && !group_all(1 + pst, 128, mbar_wait(&bars.kempty[pst], (uint32_t)((u - 1) & 1), status, 310)))
+                break;
             if (c + 2 < nch) nxt = my_row_src(gcof(c + 2));
             if (!(pre && c == pst)) fill(gcof(c), my_src);
         }
@@ -766,7 +851,7 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
         if (e != cudaSuccess) return e;
         return launch_k(attend_f32_kernel, dim3((unsigned)queries), dim3(256), smem, s, pdl, a, status);
     }
-    CUtensorMap mq, mc, mw;
+    CUtensorMap mq, mc, mw, mcr, mwr;
     if (!encode_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, kD, (uint64_t)(queries * kH), kD * 2, 64, kH,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -784,9 +869,27 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
         } else {
             mw = mc;
         }
+        mcr = mc;   // unused by the bf16 kernel
+        mwr = mc;
     } else {
-        mc = mq;   // unused by the FP8 kernel
-        mw = mq;
+        // FP8 rows (656 B) as bytes: the 512 codes in boxes of 64 rows x 64 B (no swizzle),
+        // the RoPE dims (bf16, bytes 512-639) in boxes of 64 rows x 128 B (128-byte swizzle)
+        if (a.B * a.N_c >= (int64_t(1) << 31) || a.B * a.Tw >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+        if (!encode_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.comp, 656, (uint64_t)(a.B * a.N_c), 656, 64,
+                            kChunk, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode_tmap_2d(&mcr, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.comp, 656, (uint64_t)(a.B * a.N_c), 656, 128,
+                            kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        if (a.Tw > 0) {
+            if (!encode_tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.win, 656, (uint64_t)(a.B * a.Tw), 656, 64,
+                                kChunk, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                !encode_tmap_2d(&mwr, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.win, 656, (uint64_t)(a.B * a.Tw), 656, 128,
+                                kChunk, CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        } else {
+            mw = mc;
+            mwr = mcr;
+        }
     }
     auto kern = (a.kv_dtype == LCS_KV_FP8) ? attend_tc_kernel<true> : attend_tc_kernel<false>;
     cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), kAtSmem);
@@ -798,7 +901,7 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
         part_o = static_cast<float*>(scratch);
         part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256(queries * splits * kH * kDv * 4));
     }
-    e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, mc, mw, a, splits,
+    e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, mc, mw, mcr, mwr, a, splits,
                  part_o, part_ml, status);
     if (e != cudaSuccess || splits == 1) return e;
     return launch_k(attend_combine_kernel, dim3((unsigned)(queries * kH)), dim3(128), 0, s, true, part_o, part_ml,

@@ -5,6 +5,7 @@ tiles and a ragged tail.  Tolerances: integer / byte / index work bit-exact;
 fp32 outputs max-abs 1e-4; bf16 / FP8 outputs max-abs 2e-2 x RMS(oracle).
 """
 import math
+import zlib
 
 import numpy as np
 import pytest
@@ -243,7 +244,7 @@ def test_attend_f32_c1(L, orc):
 
 
 def _rand_sel(name, B, Q, k, navail):
-    rng = np.random.default_rng(abs(hash(name)) % 2 ** 32)
+    rng = np.random.default_rng(zlib.crc32(name.encode()))   # str hash() is salted per process
     idx = np.full((B, Q, k), -1, np.int32)
     for b in range(B):
         for q in range(Q):
@@ -320,6 +321,93 @@ def test_hca_attend_decode_fp8(L, orc):
     for b in range(B):
         o, _ = orc.hca_attend(q[b, 0].double().numpy(), comp_d[b], 128, win_d[b], 0, -1, 128, dv, scale)
         assert_close_rel_rms(out[b, 0], o, 2e-2, f"hca fp8 b {b}")
+
+
+@pytest.mark.parametrize("case", ["hca_full_chunks", "csa_gathered", "hca_partial_chunks"])
+def test_attend_fp8_widening_exact(L, orc, case):
+    """FP8 rows reach the tensor cores exactly widened to bf16.  With q = 0 every score is 0,
+    every softmax weight exactly 1; every row is the same row and the number of rows is a
+    power of two, so o = V of that row, bit for bit, in fp32.  The row holds all 254
+    finite E4M3 codes (subnormals, +-0 included) under block scales 2^-117, 2^-3, 2^15 and
+    2^20.  Cases: whole 64-row chunks (TMA, widened in shared memory), gathered selected
+    rows, partial chunks (row-by-row loads)."""
+    H, D, dv = 64, 576, 512
+    codes = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    codes = np.array((codes * 3)[:512], np.uint8)
+    rope = torch.from_numpy(synth_normal("g.fp8x.r", (64,))).to(torch.bfloat16).view(torch.int16).numpy()
+    scales = np.array([2.0 ** -117, 2.0 ** -3, 2.0 ** 15, 2.0 ** 20], np.float32)
+    row = np.concatenate([codes, rope.view(np.uint8), scales.view(np.uint8)])
+    assert row.size == 656
+    n_c, tw, idx = {"hca_full_chunks": (64, 64, None), "csa_gathered": (100, 64, list(range(3, 67))),
+                    "hca_partial_chunks": (37, 27, None)}[case]
+    comp = torch.from_numpy(np.tile(row, (1, n_c, 1))).to(DEV)
+    win = torch.from_numpy(np.tile(row, (1, tw, 1))).to(DEV)
+    q = torch.zeros((1, 1, H, D), dtype=torch.bfloat16, device=DEV)   # every score exactly 0
+    if idx is None:
+        out = L.hca_attend(q, comp, win, dv, 1 / 24, kv_dtype=L.KV_FP8, out_dtype=torch.float32)
+    else:
+        sel = torch.tensor(idx, dtype=torch.int32).view(1, 1, -1).to(DEV)
+        out = L.csa_attend(q, comp, win, sel, dv, 1 / 24, kv_dtype=L.KV_FP8, out_dtype=torch.float32)
+    want = orc.dequant_kv_fp8(row)[:dv]
+    got = out[0, 0].double().cpu().numpy()
+    bad = np.nonzero(got != want[None, :])
+    assert bad[0].size == 0, f"{bad[0].size} outputs differ, first at head {bad[0][0]} dim {bad[1][0]}: " \
+                             f"{got[bad[0][0], bad[1][0]]!r} vs {want[bad[1][0]]!r}"
+
+
+def synth_normal(name, shape):
+    from long_context_sparse_06_b200 import synth
+    return synth.normal(name, shape).astype(np.float32)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_attend_rows_outside_range_unread(L, orc, kv):
+    """Rows outside a query's row set (compressed entries >= n_avail, window rows outside
+    [t-W+1, t], rows a partial 64-row chunk spans past its end) may hold anything: a cache
+    fills as the sequence grows.  Here they are all NaN; HCA and CSA must still equal the
+    oracle on the defined rows (partial window chunks of 6 and 21 rows, compressed tails
+    of 37, 37 and 8 rows)."""
+    from long_context_sparse_06_b200 import synth
+    B, H, D, dv, Nc, Tw, W, m, k = 3, 64, 576, 512, 260, 128, 128, 128, 96
+    scale = 1 / math.sqrt(576)
+    avail, nwin = [37, 101, 200], [70, 128, 21]
+    t = [m * a + 5 for a in avail]                     # n_avail = floor((t+1)/m) = avail
+    wp0 = [t[b] - (nwin[b] - 1) for b in range(B)]     # window rows 0..nwin-1 in range
+    q = randn(f"g.nan.{kv}.q", (B, 1, H, D), dtype=torch.bfloat16)
+    comp32 = synth.normal(f"g.nan.{kv}.c", (B, Nc, D)).astype(np.float32)
+    win32 = synth.normal(f"g.nan.{kv}.w", (B, Tw, D)).astype(np.float32)
+    if kv == "bf16":
+        comp_g = torch.from_numpy(comp32).to(torch.bfloat16)
+        win_g = torch.from_numpy(win32).to(torch.bfloat16)
+        comp_o, win_o = comp_g.double().numpy(), win_g.double().numpy()
+        poison = float("nan")
+        kvd = None
+    else:
+        comp_g = L.lcs_quant_kv_fp8(torch.from_numpy(comp32).to(DEV)).cpu()
+        win_g = L.lcs_quant_kv_fp8(torch.from_numpy(win32).to(DEV)).cpu()
+        comp_o = orc.dequant_kv_fp8(orc.quant_kv_fp8(comp32))
+        win_o = orc.dequant_kv_fp8(orc.quant_kv_fp8(win32))
+        poison = 0xFF                                  # NaN codes, NaN scales, NaN RoPE dims
+        kvd = L.KV_FP8
+    for b in range(B):
+        comp_g[b, avail[b]:] = poison
+        win_g[b, nwin[b]:] = poison
+    q_pos = torch.tensor(t, dtype=torch.int64).reshape(B, 1).to(DEV)
+    win_pos0 = torch.tensor(wp0, dtype=torch.int64).to(DEV)
+    qd, cd, wd = q.to(DEV), comp_g.to(DEV), win_g.to(DEV)
+    outh = both_outputs(lambda od: L.hca_attend(qd, cd, wd, dv, scale, kv_dtype=kvd, q_pos=q_pos, win_pos0=win_pos0,
+                                                m=m, W=W, out_dtype=od)).cpu().numpy()
+    idx = _rand_sel(f"sel.nan.{kv}", B, 1, k, [[a] for a in avail])
+    outc = both_outputs(lambda od: L.csa_attend(qd, cd, wd, torch.from_numpy(idx).to(DEV), dv, scale, kv_dtype=kvd,
+                                                q_pos=q_pos, win_pos0=win_pos0, W=W, out_dtype=od)).cpu().numpy()
+    assert np.isfinite(outh).all() and np.isfinite(outc).all()
+    for b in range(B):
+        qb = q[b, 0].double().numpy()
+        comp_b = comp_o[b, :avail[b]]
+        o, _ = orc.hca_attend(qb, comp_b, m, win_o[b], wp0[b], t[b], W, dv, scale)
+        assert_close_rel_rms(outh[b, 0], o, 2e-2, f"hca b {b}")
+        o, _ = orc.csa_attend(qb, comp_b, idx[b, 0], win_o[b, :nwin[b]], wp0[b], t[b], W, dv, scale)
+        assert_close_rel_rms(outc[b, 0], o, 2e-2, f"csa b {b}")
 
 
 @pytest.mark.parametrize("tail", [127, 50])
