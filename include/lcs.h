@@ -298,6 +298,20 @@ LCS_API int lcs_status(void* ws, cudaStream_t stream);
 /* Clears the status word (enqueued on stream). */
 LCS_API int lcs_clear_status(void* ws, cudaStream_t stream);
 
+/*
+ * Self-test of the bounded waits every pipelined kernel uses (the pages describe no
+ * such call).  Clears the status word of ws, then one CTA waits on an mbarrier that
+ * nothing completes: the wait gives up after budget_us microseconds (1..1e6) and
+ * records LCS_ERR_TIMEOUT, detail 901, in the status word; a second wait in the same
+ * CTA must then give up at once (detail 902 is not recorded: the first error stays).
+ * The kernel returns normally and the context stays usable.
+ *   ws   device workspace (>= 256 bytes, 256-byte aligned)
+ *   out  4 device int64: [first wait succeeded (0/1), its ns, second wait succeeded, its ns]
+ * Returns LCS_ERR_INVALID for bad arguments, LCS_ERR_CUDA without a device; the
+ * results are in ws and out once the stream reaches the kernel.
+ */
+LCS_API int lcs_selftest_wait(int budget_us, void* ws, size_t ws_bytes, long long* out, cudaStream_t stream);
+
 /* Static description of a status code. */
 LCS_API const char* lcs_error_string(int code);
 

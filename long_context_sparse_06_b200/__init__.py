@@ -16,12 +16,15 @@ __all__ = [
     "F32", "BF16", "KV_FP8", "FP4", "MODE_CSA", "MODE_HCA", "LcsError", "lib",
     "csa_compress", "hca_compress", "csa_index_topk", "lcs_topk", "csa_attend", "hca_attend",
     "decode_fused", "group_oproj", "lcs_rope", "lcs_quant_kv_fp8", "lcs_quant_fp4",
-    "lcs_workspace_size", "lcs_status", "lcs_clear_status", "workspace", "kv_fp8_row_bytes",
+    "lcs_workspace_size", "lcs_status", "lcs_clear_status", "lcs_selftest_wait", "workspace", "kv_fp8_row_bytes",
 ]
 
 F32, BF16, KV_FP8, FP4 = 0, 1, 2, 3
 MODE_CSA, MODE_HCA = 0, 1
 OP_INDEX_TOPK, OP_ATTEND, OP_DECODE, OP_TOPK = 1, 2, 3, 4
+# return codes (include/lcs.h)
+LCS_OK, LCS_ERR_INVALID, LCS_ERR_UNSUPPORTED, LCS_ERR_CUDA = 0, -1, -2, -3
+LCS_ERR_TIMEOUT, LCS_ERR_DEVICE, LCS_ERR_WORKSPACE, LCS_ERR_TOO_LARGE = -4, -5, -6, -7
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcs.so")
 
@@ -59,6 +62,7 @@ def lib():
             "lcs_quant_fp4": [P, I64, I, P, P],
             "lcs_status": [P, P],
             "lcs_clear_status": [P, P],
+            "lcs_selftest_wait": [I, P, SZ, P, P],
             "lcs_set_stage_events": [P, I],
         }
         for name, args in sig.items():
@@ -132,6 +136,11 @@ def lcs_status(ws, stream=None):
 
 def lcs_clear_status(ws, stream=None):
     _call("lcs_clear_status", _ptr(ws), _stream(stream))
+
+
+def lcs_selftest_wait(budget_us, ws, out, stream=None):
+    """Runs the bounded-wait self-test; out is a 4-element int64 device tensor."""
+    _call("lcs_selftest_wait", int(budget_us), _ptr(ws), ws.numel() * ws.element_size(), _ptr(out), _stream(stream))
 
 
 # ---------------------------------------------------------------- compressor

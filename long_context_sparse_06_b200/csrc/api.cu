@@ -209,6 +209,14 @@ int lcs_clear_status(void* ws, cudaStream_t stream) {
     return from_cuda(cudaMemsetAsync(ws, 0, kStatusBytes, stream));
 }
 
+int lcs_selftest_wait(int budget_us, void* ws, size_t ws_bytes, long long* out, cudaStream_t stream) {
+    if (ws == nullptr || out == nullptr || ws_bytes < (size_t)kStatusBytes) return LCS_ERR_INVALID;
+    if (budget_us < 1 || budget_us > 1000000) return LCS_ERR_INVALID;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return LCS_ERR_CUDA;
+    return from_cuda(launch_selftest_wait((uint64_t)budget_us * 1000ull, static_cast<int*>(ws), out, stream));
+}
+
 int lcs_status(void* ws, cudaStream_t stream) {
     if (ws == nullptr) return LCS_ERR_INVALID;
     if (!device_ok()) return LCS_ERR_CUDA;

@@ -80,24 +80,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Bounds a polling loop: every 64 polls, gives up (false) once the grid's status word
+// is non-zero or the budget is spent (recording LCS_ERR_TIMEOUT with `where`).  The
+// status word is read one check ahead of its use, so the load completes while the
+// caller polls and a wait that is about to succeed never sits behind a memory round trip.
+struct WaitBudget {
+    uint64_t t0, budget_ns;
+    uint32_t polls = 0;
+    int seen = 0;
+    __device__ __forceinline__ explicit WaitBudget(uint64_t ns = kWaitBudgetNs) : t0(globaltimer()), budget_ns(ns) {}
+    __device__ __forceinline__ bool ok(int* status, int where) {
+        if ((++polls & 63u) != 0) return true;
+        if (seen != 0) return false;
+        if (status != nullptr) seen = *(volatile int*)status;
+        if (globaltimer() - t0 > budget_ns) {
+            set_status(status, LCS_ERR_TIMEOUT, where);
+            return false;
+        }
+        return true;
+    }
+};
+
 // Waits for the phase with the given parity to complete.  Returns false (and
 // records LCS_ERR_TIMEOUT with `where` as detail) if it does not within the
 // budget.  Once any wait in the grid has failed (status non-zero) later waits
-// give up at their next check so that every thread reaches its exit path.  The
-// clock and the status word (global memory) are consulted only every 64 polls,
-// so that a wait that is about to succeed is never held up by a memory round trip.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int where) {
+// give up at a following check so that every thread reaches its exit path.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int where,
+                                          uint64_t budget_ns = kWaitBudgetNs) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
+    WaitBudget wb(budget_ns);
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (status != nullptr && *(volatile int*)status != 0) return false;
-            if (globaltimer() - t0 > kWaitBudgetNs) {
-                set_status(status, LCS_ERR_TIMEOUT, where);
-                return false;
-            }
-        }
+        if (!wb.ok(status, where)) return false;
     }
 }
 

@@ -101,4 +101,7 @@ bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, 
                     uint64_t outer2, uint64_t row_stride_bytes, uint64_t plane_stride_bytes, uint32_t box_inner,
                     uint32_t box_rows);
 
+// Bounded-wait self-test (selftest.cu): one CTA waits on an mbarrier nothing completes.
+cudaError_t launch_selftest_wait(uint64_t budget_ns, int* status, long long* out, cudaStream_t stream);
+
 }  // namespace lcs
