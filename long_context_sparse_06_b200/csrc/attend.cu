@@ -95,15 +95,23 @@ __device__ __forceinline__ bool group_all(int id, int count, bool v) {
     return r != 0;
 }
 
-// 16 E4M3 codes (a uint4, low byte first) times the power-of-two block scale s -> 16 bf16,
-// exact: code -> fp32 is exact, the product with a power of two is exact in fp32 and
-// representable in bf16, so the final rounding changes nothing.
+// Two E4M3 codes (low byte first) times the power-of-two block scale s -> two bf16, exact:
+// one conversion instruction per pair to f16 (exact: every E4M3 value is a normal f16),
+// f16 -> fp32 exact, the product with a power of two exact in fp32 and representable in
+// bf16, so the final rounding changes nothing.
+__device__ __forceinline__ uint32_t widen_e4m3x2(uint32_t two, float s) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<__half2*>(&h));
+    return pack_bf16x2(f.x * s, f.y * s);
+}
+
+// 16 E4M3 codes (a uint4, low byte first) -> 16 bf16 (8 packed pairs).
 __device__ __forceinline__ void widen16(uint4 v, float s, uint32_t (&o)[8]) {
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        o[2 * q] = pack_bf16x2(e4m3_to_f32(w4[q] & 0xFF) * s, e4m3_to_f32((w4[q] >> 8) & 0xFF) * s);
-        o[2 * q + 1] = pack_bf16x2(e4m3_to_f32((w4[q] >> 16) & 0xFF) * s, e4m3_to_f32(w4[q] >> 24) * s);
+        o[2 * q] = widen_e4m3x2(w4[q], s);
+        o[2 * q + 1] = widen_e4m3x2(w4[q] >> 16, s);
     }
 }
 
