@@ -430,7 +430,7 @@ ORC_API void orc_index_scores_bf16(const double* qI, const float* w, const doubl
  * q_packed/q_scales: the query quantised by orc_quant_fp4 ([H, dI]). */
 ORC_API void orc_index_scores_fp4(const uint8_t* q_packed, const uint8_t* q_scales, const float* w,
                                   const uint8_t* k_packed, const uint8_t* k_scales, int64_t N,
-                                  int H, int dI, double* score_bf16)
+                                  int H, int dI, int round_bf16, double* score)
 {
     int nb = dI / 32;
     for (int64_t s = 0; s < N; ++s) {
@@ -454,7 +454,8 @@ ORC_API void orc_index_scores_fp4(const uint8_t* q_packed, const uint8_t* q_scal
             float r = dot > 0.0f ? dot : 0.0f;
             acc = fmaf(w[h], r, acc);
         }
-        score_bf16[s] = orc_round_bf16((double)acc);
+        /* the pages' BF16 index score; the fp32 sum itself when round_bf16 == 0 */
+        score[s] = round_bf16 ? orc_round_bf16((double)acc) : (double)acc;
     }
 }
 

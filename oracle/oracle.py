@@ -67,7 +67,7 @@ def lib():
             "orc_compress": (I, [P, P, P, P, P, I64, I, I, I, I, D, I64, P, P]),
             "orc_index_scores_f32": (None, [P, P, P, I64, I, I, P]),
             "orc_index_scores_bf16": (None, [P, P, P, I64, I, I, P]),
-            "orc_index_scores_fp4": (None, [P, P, P, P, P, I64, I, I, P]),
+            "orc_index_scores_fp4": (None, [P, P, P, P, P, I64, I, I, I, P]),
             "orc_exact_dot_f32": (C.c_float, [P, P, I]),
             "orc_topk": (None, [P, I64, I, P]),
             "orc_mqa_rows": (None, [P, P, I64, I, I, I, D, P, P]),
@@ -241,15 +241,17 @@ def index_scores_bf16(qI, w, kI):
     return out
 
 
-def index_scores_fp4(qI, w, k_packed, k_scales):
+def index_scores_fp4(qI, w, k_packed, k_scales, round_bf16=True):
     """FP4 QK path ("DeepSeek V4 深度解析" §4; "V3 vs V4" page "FP4 为什么能无损"):
-    qI [H, dI] (bf16 values) is quantised like the keys; scores rounded to bf16."""
+    qI [H, dI] (bf16 values) is quantised like the keys; scores rounded to bf16 (the
+    same page: index scores in BF16), or the fp32 sum before that rounding."""
     qp, qs = quant_fp4(_f32(qI))
     w = _f32(w)
     kp, ks = np.ascontiguousarray(k_packed, np.uint8), np.ascontiguousarray(k_scales, np.uint8)
     H, dI = np.asarray(qI).shape
     out = np.empty(kp.shape[0], np.float64)
-    lib().orc_index_scores_fp4(_p(qp), _p(qs), _p(w), _p(kp), _p(ks), kp.shape[0], H, dI, _p(out))
+    lib().orc_index_scores_fp4(_p(qp), _p(qs), _p(w), _p(kp), _p(ks), kp.shape[0], H, dI, int(bool(round_bf16)),
+                               _p(out))
     return out
 
 

@@ -334,6 +334,12 @@ def test_index_fp4_against_dequantised_fp64(orc):
     bound = np.maximum(np.abs(dots), 0) @ np.abs(w) * (H + 6) * 2.0 ** -23 + np.abs(ref) * 2.0 ** -8 + 1e-30
     assert np.all(np.abs(s - ref) <= bound)
     np.testing.assert_array_equal(orc.round_bf16(s), s)
+    # the fp32 sum before the bf16 rounding: the fp32 chain error alone
+    s32 = orc.index_scores_fp4(qI, w, kp, ks, round_bf16=False)
+    bound32 = np.maximum(np.abs(dots), 0) @ np.abs(w) * (H + 6) * 2.0 ** -23 + 1e-30
+    assert np.all(np.abs(s32 - ref) <= bound32)
+    np.testing.assert_array_equal(s32.astype(np.float32).astype(np.float64), s32)
+    np.testing.assert_array_equal(orc.round_bf16(s32), s)
     # the block dots are exact multiples of 1/4 (checked through a one-block key)
     one = np.zeros((1, dI), np.float32); one[0, :32] = kraw[0, :32]
     p1, s1 = orc.quant_fp4(one)
