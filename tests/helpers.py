@@ -24,6 +24,28 @@ def assert_close_rel_rms(got, ref, rel=2e-2, what=""):
     return err, bound
 
 
+def bf16_half_ulp(x):
+    """Half a bf16 ulp at |x| (bf16 keeps 8 significant bits): the most that storing a
+    value of that size in bf16 with round-to-nearest-even can move it."""
+    x = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(x, 2.0 ** -126)))
+    return 2.0 ** (e - 8)
+
+
+def assert_close_stored_bf16(got, ref, rel=2e-2, what=""):
+    """Outputs stored in bf16: the kernel's value lies within rel * RMS(ref) of the oracle,
+    and storing it rounds it by at most half a bf16 ulp (round-to-nearest-even), so each
+    element lies within rel * RMS(ref) + half an ulp at |ref| + rel * RMS(ref)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    slack = rel * rms(ref)
+    bound = slack + bf16_half_ulp(np.abs(ref) + slack)
+    excess = np.abs(got - ref) - bound
+    i = int(np.argmax(excess)) if excess.size else 0
+    assert excess.size == 0 or excess.flat[i] <= 0, \
+        f"{what}: error {abs(got.flat[i] - ref.flat[i]):.3e} at |ref| {abs(ref.flat[i]):.3e} > {bound.flat[i]:.3e}"
+
+
 def assert_close_abs(got, ref, tol=1e-4, what=""):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
@@ -39,3 +61,37 @@ def topk_gap_ok(oracle_scores, k, bound):
     if s.size <= k:
         return True
     return (s[k - 1] - s[k]) > 2 * bound
+
+
+def bf16_score_bound(qI, w, kI):
+    """|GPU - oracle| bound per key for bf16 index scores: each per-head dot from the
+    tensor cores carries at most (d_I/16 + 1) fp32 roundings (or truncations) of partial
+    sums bounded by sum|q||k|; the head chain adds H roundings."""
+    qa, ka = np.abs(qI), np.abs(kI)
+    sabs = ka @ qa.T                                   # [N, H]
+    dI = qI.shape[1]
+    dot_err = (dI // 16 + 1) * 2.0 ** -23 * sabs
+    relu_abs = sabs                                    # |relu(dot)| <= sum|q||k|
+    return dot_err @ np.abs(w) * 1.01 + relu_abs @ np.abs(w) * (w.size + 2) * 2.0 ** -24
+
+
+def assert_exact_topk(scores, idx, k, what=""):
+    """idx (ascending, -1 padded) selects the k largest of `scores` by (score desc, index
+    asc): a property of any size, checked on the scores the kernels computed."""
+    s = np.asarray(scores, np.float32)
+    idx = np.asarray(idx)
+    n = s.size
+    t = min(k, n)
+    sel = idx[:t]
+    assert np.all(idx[t:] == -1), f"{what}: padding"
+    assert sel.size == 0 or (np.all(np.diff(sel) > 0) and sel.min() >= 0 and sel.max() < n), f"{what}: order/range"
+    if t == n or t == 0:
+        return
+    mask = np.zeros(n, bool)
+    mask[sel] = True
+    v = s[sel].min()
+    assert s[~mask].max() <= v, f"{what}: an unselected score exceeds the selection's minimum"
+    tie_uns = np.nonzero(~mask & (s == v))[0]
+    if tie_uns.size:
+        tie_sel = sel[s[sel] == v]
+        assert tie_sel.max() < tie_uns.min(), f"{what}: a tie at the threshold went to a higher index"

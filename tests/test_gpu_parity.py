@@ -12,6 +12,7 @@ import pytest
 import torch
 
 from helpers import assert_close_abs, assert_close_rel_rms, randn, topk_gap_ok
+from helpers import bf16_score_bound as _bf16_score_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -159,18 +160,6 @@ def test_index_f32_bit_exact(L, orc):
         ref = orc.index_scores_f32(qI[0, q].numpy(), w[0, q].numpy(), kI[0, :n].numpy())
         np.testing.assert_array_equal(sc[0, q, :n], ref)
         np.testing.assert_array_equal(idx[0, q], orc.topk(ref, k))
-
-
-def _bf16_score_bound(qI, w, kI):
-    """|GPU - oracle| bound for bf16 scores: each per-head dot from the tensor
-    cores carries at most (d_I/16 + 1) fp32 roundings (or truncations) of partial
-    sums bounded by sum|q||k|; the head chain adds H roundings."""
-    qa, ka = np.abs(qI), np.abs(kI)
-    sabs = ka @ qa.T                                   # [N, H]
-    dI = qI.shape[1]
-    dot_err = (dI // 16 + 1) * 2.0 ** -23 * sabs
-    relu_abs = sabs                                    # |relu(dot)| <= sum|q||k|
-    return dot_err @ np.abs(w) * 1.01 + relu_abs @ np.abs(w) * (w.size + 2) * 2.0 ** -24
 
 
 def test_index_bf16_tensor_cores(L, orc):
