@@ -174,8 +174,9 @@ LCS_API int lcs_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, 
  * Tensor-core paths: H == 64, D == 576, d_v == 512.  F32 path: H <= 64, D <= 128.
  * Only rows of R contribute: rows of comp and win outside R may hold anything, NaN
  * included (a cache that fills as the sequence grows).  Tensor-core paths load runs of
- * consecutive rows by TMA: comp and win start on a 16-byte boundary, and B*N_c, B*Tw
- * stay below 2^31 (else LCS_ERR_CUDA and the attention is not launched).
+ * consecutive rows by TMA: comp and win start on a 16-byte boundary (else
+ * LCS_ERR_INVALID), and B*N_c, B*Tw stay below 2^31 (else LCS_ERR_UNSUPPORTED); both
+ * are checked before anything is enqueued.
  */
 LCS_API int csa_attend(const void* q, int q_dtype, const void* comp, const void* win, int kv_dtype,
                int64_t B, int64_t Q, int64_t N_c, int64_t Tw, const int32_t* idx, int k,

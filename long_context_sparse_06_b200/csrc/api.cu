@@ -349,6 +349,8 @@ static int validate_attend(const AttendArgs& a, int q_dtype, int out_dtype) {
     if (a.kv_dtype == LCS_BF16 || a.kv_dtype == LCS_KV_FP8) {
         if (q_dtype != LCS_BF16 || (out_dtype != LCS_BF16 && out_dtype != LCS_F32)) return LCS_ERR_UNSUPPORTED;
         if (a.H != 64 || a.D != 576 || a.d_v != 512 || a.k > 2048) return LCS_ERR_UNSUPPORTED;
+        // runs of consecutive rows are loaded by TMA, whose row coordinates are int32
+        if (a.B * a.N_c >= (int64_t(1) << 31) || a.B * a.Tw >= (int64_t(1) << 31)) return LCS_ERR_UNSUPPORTED;
         if (!aligned16(a.q) || !aligned16(a.comp) || (a.win && !aligned16(a.win)) || !aligned16(a.out))
             return LCS_ERR_INVALID;
         return LCS_OK;

@@ -57,6 +57,16 @@ def test_validation_without_device(L):
                           None, P, 1 << 20, None) == -2
     assert lib.hca_attend(P, L.BF16, P, None, L.BF16, 1, 1, 10, 4, None, None, 128, 128, 64, 576, 512, 0.1, P,
                           L.BF16, None, P, 1 << 20, None) == -1
+    # row buffers off a 16-byte boundary (TMA); more rows than int32 row coordinates reach
+    for kv in (L.BF16, L.KV_FP8):
+        assert lib.hca_attend(P, L.BF16, P + 8, P, kv, 1, 1, 10, 4, None, None, 128, 128, 64, 576, 512, 0.1, P,
+                              L.BF16, None, P, 1 << 20, None) == -1
+        assert lib.hca_attend(P, L.BF16, P, P + 8, kv, 1, 1, 10, 4, None, None, 128, 128, 64, 576, 512, 0.1, P,
+                              L.BF16, None, P, 1 << 20, None) == -1
+        assert lib.hca_attend(P, L.BF16, P, P, kv, 2, 1, 1 << 30, 4, None, None, 128, 128, 64, 576, 512, 0.1, P,
+                              L.BF16, None, P, 1 << 20, None) == -2
+        assert lib.csa_attend(P, L.BF16, P, P, kv, 1 << 20, 1, 1 << 11, 4, P, 4, None, None, 128, 64, 576, 512, 0.1,
+                              P, L.BF16, None, P, 1 << 20, None) == -2
     assert lib.decode_fused(5, 1, P, L.BF16, P, P, L.BF16, 10, 4, 64, 576, 512, 0.1, P, L.BF16, P, P, L.BF16, 64, 128,
                             8, L.F32, P, L.BF16, None, None, P, 1 << 20, None) == -1
     assert lib.group_oproj(P, 4, 8, 48, P, 3, 64, P, 256, P, None) == -1
