@@ -172,6 +172,7 @@ LCS_API int lcs_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, 
  *   out  [B, Q, H, d_v] out_dtype (LCS_F32 for f32 kv, LCS_BF16 otherwise)
  *   lse  [B, Q, H]      fp32 natural-log sum of exp(scale*q.K) over R, or NULL
  * Tensor-core paths: H == 64, D == 576, d_v == 512.  F32 path: H <= 64, D <= 128.
+ * An empty R (no selected entry, no window row) gives o = 0 and lse = -inf.
  * Only rows of R contribute: rows of comp and win outside R may hold anything, NaN
  * included (a cache that fills as the sequence grows).  Tensor-core paths load runs of
  * consecutive rows by TMA: comp and win start on a 16-byte boundary (else

@@ -399,6 +399,48 @@ def test_attend_rows_outside_range_unread(L, orc, kv):
         assert_close_rel_rms(outc[b, 0], o, 2e-2, f"csa b {b}")
 
 
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_attend_degenerate_row_sets(L, orc, kv):
+    """Degenerate row sets: a selection that is all -1 (the window alone), no window at
+    all (Tw = 0: the selection alone), and neither (R empty: o = 0, lse = -inf)."""
+    from long_context_sparse_06_b200 import synth
+    B, H, D, dv, Nc, k, Tw = 2, 64, 576, 512, 700, 200, 128
+    scale = 1 / 24
+    q = randn(f"g.dg.{kv}.q", (B, 1, H, D), dtype=torch.bfloat16)
+    comp32 = synth.normal(f"g.dg.{kv}.c", (B, Nc, D)).astype(np.float32)
+    win32 = synth.normal(f"g.dg.{kv}.w", (B, Tw, D)).astype(np.float32)
+    if kv == "bf16":
+        comp_g, win_g = torch.from_numpy(comp32).to(torch.bfloat16), torch.from_numpy(win32).to(torch.bfloat16)
+        comp_o, win_o = comp_g.double().numpy(), win_g.double().numpy()
+        comp_g, win_g, kvd = comp_g.to(DEV), win_g.to(DEV), None
+    else:
+        comp_g = L.lcs_quant_kv_fp8(torch.from_numpy(comp32).to(DEV))
+        win_g = L.lcs_quant_kv_fp8(torch.from_numpy(win32).to(DEV))
+        comp_o = orc.dequant_kv_fp8(orc.quant_kv_fp8(comp32))
+        win_o = orc.dequant_kv_fp8(orc.quant_kv_fp8(win32))
+        kvd = L.KV_FP8
+    qd = q.to(DEV)
+    sel = _rand_sel(f"sel.dg.{kv}", B, 1, k, Nc)
+    none = np.full((B, 1, k), -1, np.int32)
+    no_win = np.zeros((0, D))
+    # the window alone
+    out = both_outputs(lambda od: L.csa_attend(qd, comp_g, win_g, torch.from_numpy(none).to(DEV), dv, scale,
+                                               kv_dtype=kvd, out_dtype=od)).cpu().numpy()
+    for b in range(B):
+        o, _ = orc.csa_attend(q[b, 0].double().numpy(), comp_o[b], none[b, 0], win_o[b], 0, -1, 128, dv, scale)
+        assert_close_rel_rms(out[b, 0], o, 2e-2, f"window alone b {b}")
+    # the selection alone
+    out = both_outputs(lambda od: L.csa_attend(qd, comp_g, None, torch.from_numpy(sel).to(DEV), dv, scale,
+                                               kv_dtype=kvd, out_dtype=od)).cpu().numpy()
+    for b in range(B):
+        o, _ = orc.csa_attend(q[b, 0].double().numpy(), comp_o[b], sel[b, 0], no_win, 0, -1, 128, dv, scale)
+        assert_close_rel_rms(out[b, 0], o, 2e-2, f"selection alone b {b}")
+    # nothing: the empty sum
+    out, lse = L.csa_attend(qd, comp_g, None, torch.from_numpy(none).to(DEV), dv, scale, kv_dtype=kvd,
+                            want_lse=True, out_dtype=torch.float32)
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
 @pytest.mark.parametrize("tail", [127, 50])
 def test_attend_prefill_tc_causal(L, orc, tail):
     """C4-shaped (smaller): queries at positions p0.., window from the chunk plus a prefix tail

@@ -451,6 +451,22 @@ def test_attention_closed_forms(orc):
     np.testing.assert_allclose(o, (1 - p1)[:, None] * r2[0, :dv] + p1[:, None] * r2[1, :dv], rtol=0, atol=1e-14)
 
 
+def test_attention_empty_row_set(orc):
+    """No selected entry and no window row: the empty sum, o = 0 and lse = log 0 = -inf,
+    whether the set is empty by selection (-1 padding) or by an empty window."""
+    D, dv = 576, 512
+    q = synth.normal("pin.em.q", (4, D))
+    comp = synth.normal("pin.em.c", (10, D))
+    none = np.full(8, -1, np.int32)
+    o, l = orc.csa_attend(q, comp, none, np.zeros((0, D)), 0, -1, 128, dv, 0.1)
+    np.testing.assert_array_equal(o, np.zeros((4, dv)))
+    assert np.all(np.isneginf(l))
+    win = synth.normal("pin.em.w", (6, D))                    # window rows all after the query
+    o, l = orc.csa_attend(q, comp, none, win, 100, 50, 128, dv, 0.1)
+    np.testing.assert_array_equal(o, np.zeros((4, dv)))
+    assert np.all(np.isneginf(l))
+
+
 def test_group_oproj_equals_block_diagonal(orc):
     from scipy.linalg import block_diag
     H, dv, G, dg, hidden = 8, 48, 2, 64, 256
