@@ -221,6 +221,68 @@ def compress(x, z, bias, m, overlap, d_rope=0, theta=10000.0, pos0=0, x_tail=Non
     return out, pw
 
 
+# ----------------------------------------------------- decode-time cache update
+class CacheState:
+    """One request's caches as tokens arrive one at a time ("DeepSeek V4 深度解析" §4, the
+    KV cache for mixed attention): a state cache holding the sliding window's rows and the
+    raw tail not yet enough to compress, and a compressed cache of CSA and HCA entries in
+    blocks that each cover lcm(m, m') raw tokens.
+
+    append() takes token t's raw (un-rotated) KV row x, its index-key row kx and its three
+    pooling logits; an entry is emitted as soon as its last token has arrived, pooled
+    exactly as the whole-sequence compressor pools it.  The window keeps the last W rows
+    after RoPE at their own positions (the rows attention reads)."""
+
+    def __init__(self, bias, biasI, biash, d_rope, m=4, overlap=2, mh=128, W=128, theta=10000.0):
+        self.bias, self.biasI, self.biash = _f64(bias), _f64(biasI), _f64(biash)
+        self.d_rope, self.m, self.overlap, self.mh, self.W, self.theta = d_rope, m, overlap, mh, W, theta
+        self.t = 0
+        self.raw, self.kraw, self.z, self.zI, self.zh = [], [], [], [], []   # the uncompressed tails
+        self.window = []                                                      # (position, rotated row)
+        self.csa, self.csa_keys, self.hca = [], [], []
+
+    def append(self, x, kx, z, zI, zh):
+        t = self.t
+        x, kx = _f64(x), _f64(kx)
+        self.raw.append(x)
+        self.kraw.append(kx)
+        self.z.append(float(z))
+        self.zI.append(float(zI))
+        self.zh.append(float(zh))
+        self.window.append((t, rope(x[None], t, self.d_rope, self.theta)[0]))
+        self.window = self.window[-self.W:]
+        m, ov = self.m, self.overlap
+        if (t + 1) % m == 0:                       # CSA entry j = t // m: tokens m*j - ov .. t
+            j = t // m
+            have = min(ov, m * j)                  # overlap rows that exist before the entry
+            rows = np.array(self.raw[-(m + have):])
+            krows = np.array(self.kraw[-(m + have):])
+            zz, zzI = np.array(self.z[-(m + have):]), np.array(self.zI[-(m + have):])
+            tail = (rows[:have], zz[:have]) if have else (None, None)
+            ktail = (krows[:have], zzI[:have]) if have else (None, None)
+            e, _ = compress(rows[have:], zz[have:], self.bias, m, ov, self.d_rope, self.theta, m * j, tail[0], tail[1])
+            k, _ = compress(krows[have:], zzI[have:], self.biasI, m, ov, 0, self.theta, m * j, ktail[0], ktail[1])
+            self.csa.append(e[0])
+            self.csa_keys.append(k[0])
+        if (t + 1) % self.mh == 0:                 # HCA entry h = t // mh: tokens mh*h .. t
+            h = t // self.mh
+            rows = np.array(self.raw[-self.mh:])
+            zz = np.array(self.zh[-self.mh:])
+            e, _ = compress(rows, zz, self.biash, self.mh, 0, self.d_rope, self.theta, self.mh * h)
+            self.hca.append(e[0])
+        # the tail keeps what the next entries still need: the overlap rows and the rows of
+        # the incomplete CSA entry, and the rows of the incomplete HCA entry
+        keep = max(ov + (t + 1) % m, (t + 1) % self.mh)
+        self.raw, self.kraw = self.raw[-keep:] if keep else [], self.kraw[-keep:] if keep else []
+        self.z, self.zI, self.zh = (self.z[-keep:] if keep else [], self.zI[-keep:] if keep else [],
+                                    self.zh[-keep:] if keep else [])
+        self.t = t + 1
+
+    def blocks(self):
+        """Complete compressed-cache blocks: each covers lcm(m, m') raw tokens."""
+        return self.t // np.lcm(self.m, self.mh)
+
+
 # ---------------------------------------------------------------- indexer
 def index_scores_f32(qI, w, kI):
     """fp32 lightning-indexer scores in the fixed fma order ("DeepSeek V4 深度解析" §2 step 2).

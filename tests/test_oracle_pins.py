@@ -467,6 +467,41 @@ def test_attention_empty_row_set(orc):
     assert np.all(np.isneginf(l))
 
 
+@pytest.mark.parametrize("T", [300, 130])
+def test_cache_stream_equals_whole_sequence(orc, T):
+    """Tokens appended one at a time emit, as each entry completes, exactly the entries the
+    whole-sequence compressor makes (CSA KV, CSA index keys, HCA KV); the state cache then
+    holds the uncompressed tail and the last W rows after RoPE at their own positions; the
+    compressed cache holds whole blocks of lcm(4, 128) = 128 raw tokens."""
+    D, DI, dr, W = 64, 32, 16, 128
+    x = synth.normal(f"pin.cs{T}.x", (T, D))
+    kx = synth.normal(f"pin.cs{T}.k", (T, DI))
+    z, zI, zh = (synth.normal(f"pin.cs{T}.{n}", T) for n in ("z", "zI", "zh"))
+    bias, biasI = synth.normal("pin.cs.b", 6), synth.normal("pin.cs.bI", 6)
+    biash = synth.normal("pin.cs.bh", 128)
+    st = orc.CacheState(bias, biasI, biash, dr, W=W)
+    n_csa = []
+    for t in range(T):
+        st.append(x[t], kx[t], z[t], zI[t], zh[t])
+        n_csa.append(len(st.csa))
+    assert n_csa == [(t + 1) // 4 for t in range(T)]               # emitted as soon as complete
+    csa, _ = orc.compress(x[:T // 4 * 4], z[:T // 4 * 4], bias, 4, 2, dr)
+    keys, _ = orc.compress(kx[:T // 4 * 4], zI[:T // 4 * 4], biasI, 4, 2, 0)
+    nh = T // 128
+    hca, _ = orc.compress(x[:nh * 128], zh[:nh * 128], biash, 128, 0, dr)
+    np.testing.assert_array_equal(np.array(st.csa), csa)
+    np.testing.assert_array_equal(np.array(st.csa_keys), keys)
+    np.testing.assert_array_equal(np.array(st.hca).reshape(nh, D), hca)
+    pos = [p_ for p_, _ in st.window]
+    assert pos == list(range(max(0, T - W), T))
+    np.testing.assert_array_equal(np.array([r for _, r in st.window]),
+                                  orc.rope(x[max(0, T - W):], np.arange(max(0, T - W), T), dr))
+    keep = max(2 + T % 4, T % 128)
+    assert len(st.raw) == keep
+    np.testing.assert_array_equal(np.array(st.raw), x[T - keep:])
+    assert st.blocks() == T // 128 and len(st.hca) == st.blocks() and len(st.csa) >= 32 * st.blocks()
+
+
 def test_group_oproj_equals_block_diagonal(orc):
     from scipy.linalg import block_diag
     H, dv, G, dg, hidden = 8, 48, 2, 64, 256
