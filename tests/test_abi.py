@@ -86,3 +86,28 @@ def test_valid_call_without_device_fails_loudly(L):
     P = 4096
     assert lib.lcs_quant_fp4(P, 4, 64, P, None) == -3
     assert lib.csa_compress(P, L.BF16, 1, 8, 576, None, None, P, P, 4, 2, 64, 1e4, 0, P, L.BF16, None) == -3
+
+
+def _header_arg_counts():
+    """Parameter count of every declaration in include/lcs.h (comments stripped)."""
+    txt = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"LCS_API\s+(?:const\s+)?[a-z0-9_]+\**\s+\**([a-z_0-9]+)\s*\(([^)]*)\)", txt):
+        params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_signatures_match_the_header(L):
+    """Every function the Python binding declares to ctypes takes as many arguments as its
+    C declaration: a mismatch would shift every later argument silently."""
+    lib = L.lib()
+    counts = _header_arg_counts()
+    assert len(counts) == len(declared())
+    checked = 0
+    for name, n in counts.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == n, f"{name}: binding has {len(fn.argtypes)} arguments, header {n}"
+            checked += 1
+    assert checked == len(counts)          # every declared function is bound
