@@ -98,16 +98,30 @@ def _header_arg_counts():
     return out
 
 
+def _ctype_of(param):
+    """The ctypes type a C parameter declaration needs (x86-64: a 32-bit int passed for an
+    int64_t leaves the register's upper half undefined)."""
+    p = param.strip()
+    if "*" in p or p.startswith("cudaStream_t"):
+        return C.c_void_p
+    kind = p.split()[0] if not p.startswith("const ") else p.split()[1]
+    return {"int64_t": C.c_int64, "int": C.c_int, "float": C.c_float, "size_t": C.c_size_t}[kind]
+
+
 def test_binding_signatures_match_the_header(L):
-    """Every function the Python binding declares to ctypes takes as many arguments as its
-    C declaration: a mismatch would shift every later argument silently."""
+    """Every function the Python binding declares to ctypes takes the arguments of its C
+    declaration, in number and in kind: a mismatch would corrupt the call silently."""
     lib = L.lib()
     counts = _header_arg_counts()
     assert len(counts) == len(declared())
+    txt = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
     checked = 0
-    for name, n in counts.items():
+    for m in re.finditer(r"LCS_API\s+(?:const\s+)?[a-z0-9_]+\**\s+\**([a-z_0-9]+)\s*\(([^)]*)\)", txt):
+        name, params = m.group(1), [q for q in m.group(2).split(",") if q.strip() and q.strip() != "void"]
         fn = getattr(lib, name)
-        if fn.argtypes is not None:
-            assert len(fn.argtypes) == n, f"{name}: binding has {len(fn.argtypes)} arguments, header {n}"
-            checked += 1
-    assert checked == len(counts)          # every declared function is bound
+        assert fn.argtypes is not None, f"{name} is not bound"
+        assert len(fn.argtypes) == counts[name], f"{name}: binding has {len(fn.argtypes)} arguments, header {counts[name]}"
+        for i, (q, t) in enumerate(zip(params, fn.argtypes)):
+            assert t == _ctype_of(q), f"{name} argument {i} ({q.strip()}): binding {t.__name__}"
+        checked += 1
+    assert checked == len(counts)
