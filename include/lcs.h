@@ -219,7 +219,10 @@ LCS_API int hca_attend(const void* q, int q_dtype, const void* comp, const void*
  * The first call on each device looks the array up with cudaGetSymbolAddress
  * (with that device current), which may make the CUDA runtime load the
  * module that holds the array; make that first call before any stream
- * capture starts.  Returns LCS_ERR_CUDA if the lookup fails.
+ * capture starts.  The lookup is repeated when the device's context has
+ * changed since (a cudaDeviceReset destroys the context and the module with
+ * it); make the first call after such a reset before any capture as well.
+ * Returns LCS_ERR_CUDA if the lookup fails.
  * All calls on one device share the array: calls that overlap in time (other
  * streams, other host threads) race on it and must be serialised by the caller.
  */

@@ -144,3 +144,24 @@ def with_outliers_t(name: str, x, frac: float = 0.01, factor: float = 20.0, seed
     import torch
     u = uniform_t(name + ".outlier", x.numel(), seed, device=x.device).reshape(x.shape)
     return torch.where(u < frac, x * factor, x)
+
+
+def normal_rows_t(name: str, shape, rows, seed: int = 0, std: float = 1.0, dtype=None):
+    """Rows `rows` (indices along the first dim) of normal_t(name, shape), made on the host
+    without the rest of the tensor: output i of the stream depends on i alone.  The row
+    width must be even (rows then start on a Box-Muller pair)."""
+    import torch
+    shape = tuple(shape)
+    width = int(np.prod(shape[1:]))
+    assert width % 2 == 0, "row width must be even"
+    dtype = dtype or torch.float32
+    rows = torch.as_tensor(rows, dtype=torch.int64).reshape(-1)
+    key = _u64_to_i64(int(_key(name, seed)))
+    # counters of the pairs of each row: pair p uses outputs 2p+1 and 2p+2
+    p0 = rows[:, None] * (width // 2) + torch.arange(width // 2, dtype=torch.int64)[None, :]
+    c1 = (2 * p0 + 1).reshape(-1)
+    u1 = (_lsr_t(_mix_t(c1 * _GAMMA_I + key), 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    u2 = (_lsr_t(_mix_t((c1 + 1) * _GAMMA_I + key), 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    r = torch.sqrt(-2.0 * torch.log(u1))
+    z = torch.stack([r * torch.cos(2.0 * np.pi * u2), r * torch.sin(2.0 * np.pi * u2)], dim=1).reshape(-1)
+    return (z * std).to(dtype).reshape((rows.numel(),) + shape[1:])

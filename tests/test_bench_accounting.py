@@ -63,3 +63,24 @@ def test_compress_stream_bytes():
     hca = T * D * 2 + T * 4 + (T // 128) * D * 2
     assert wl.alg_bytes_per_step() == csa_kv + csa_keys + hca
     assert wl.dominant_bytes() == csa_kv
+
+
+def test_c1_attention_flops():
+    """C1: QK (64 dims) and PV (48 dims) over each query's selected entries (up to 64 of
+    its complete ones) and its causal window (up to 128 rows), 8 heads."""
+    wl = bench.C1Prefill(None, "cpu", 0)
+    sel = sum(min(64, (t + 1) // 4) for t in range(1024))
+    win = sum(min(128, t + 1) for t in range(1024))
+    assert sel == 57_280                                       # the selected (query, entry) pairs
+    assert wl.attend_flops() == (sel + win) * 8 * (64 + 48) * 2
+
+
+def test_rows_generator_matches_whole_tensor():
+    """The reference arm makes only the selected compressed rows; they equal the same rows
+    of the whole seeded tensor the GPU arm makes."""
+    import torch
+    from long_context_sparse_06_b200 import synth
+    full = synth.normal_t("acct.rows", (3, 40, 576), dtype=torch.bfloat16)
+    idx = torch.tensor([0, 39, 40, 77, 119])
+    got = synth.normal_rows_t("acct.rows", (120, 576), idx, dtype=torch.bfloat16)
+    assert torch.equal(got, full.reshape(120, 576)[idx])

@@ -1,0 +1,166 @@
+"""The tiny fp32 CSA prefill end to end: seq 1024, hidden 256, on one seeded instance.
+
+"DeepSeek V4 深度解析" §2, CSA steps 1-3 and the HCA paragraph: the KV and the index keys
+are pooled by two compressors (m = 4, overlap 2, bias of shape [6]), the lightning
+indexer (4 heads x 32) scores the entries causally and keeps the top 64, 8 query heads
+attend over the selection and the last 128 raw rows (KV dim 64 = 48 + 16 RoPE), and a
+grouped output projection (2 groups of 64) maps the heads to the hidden size.
+
+The projections from the hidden states (KV, index keys, pooling logits, index queries and
+head weights, queries) are harness inputs, computed here in fp64 and rounded to fp32; both
+sides get the same values.  Every stage is then checked against the oracle:
+  * each compressor within max-abs 1e-4;
+  * the indexer and top-k bit-exact (scores and selection) on the oracle's entries;
+  * attention and its LSE within 1e-4 on the oracle's entries and selection;
+  * the grouped projection within 1e-4 on the oracle's attention output;
+  * the whole chain run on the GPU's own intermediates: the selection equals the
+    oracle's for every query whose k-th score gap exceeds the effect of the compressors'
+    rounding, and the projected output is within 1e-4 for those queries.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close_abs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+T, HID, M, OV = 1024, 256, 4, 2
+DKV, DR, DV = 64, 16, 48
+HI, DI, K = 4, 32, 64
+H, W, G, DG = 8, 128, 2, 64
+NC = T // M
+SCALE = 1.0 / math.sqrt(DKV)
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import long_context_sparse_06_b200 as lcs
+    lcs.lib()
+    return lcs
+
+
+def _inputs():
+    """Hidden states N(0,1), weights N(0, 1/fan_in), biases N(0,1); projections in fp64,
+    rounded to fp32."""
+    from long_context_sparse_06_b200 import synth
+    r = lambda name, shape, std=1.0: synth.normal("c1." + name, shape, std=std)   # noqa: E731
+    f32 = lambda a: np.asarray(a, np.float64).astype(np.float32)                    # noqa: E731
+    h = f32(r("h", (T, HID)))
+    hd = h.astype(np.float64)
+    sw = 1.0 / math.sqrt(HID)
+    p = dict(
+        x=f32(hd @ f32(r("W_kv", (HID, DKV), sw))),
+        kx=f32(hd @ f32(r("W_ki", (HID, DI), sw))),
+        z=f32(hd @ f32(r("w_z", HID, sw))),
+        zI=f32(hd @ f32(r("w_zi", HID, sw))),
+        qI=f32(hd @ f32(r("W_qi", (HID, HI * DI), sw))).reshape(T, HI, DI),
+        w=f32(hd @ f32(r("W_w", (HID, HI), sw))),
+        q_raw=f32(hd @ f32(r("W_q", (HID, H * DKV), sw))).reshape(T, H, DKV),
+        bias=f32(r("bias", 6)),
+        biasI=f32(r("bias_i", 6)),
+        Wg=f32(r("Wg", (G, H // G * DV, DG), 1.0 / math.sqrt(H // G * DV))),
+        Wo=f32(r("Wo", (G * DG, HID), 1.0 / math.sqrt(G * DG))),
+    )
+    return p
+
+
+def _oracle_chain(orc, p, comp, kI):
+    """The oracle's indexer, top-k, attention and projection over the given entries."""
+    pos = np.arange(T)
+    win = orc.rope(p["x"].astype(np.float64), pos, DR).astype(np.float32)
+    q = orc.rope(p["q_raw"].reshape(T * H, DKV).astype(np.float64), np.repeat(pos, H), DR)
+    q = q.reshape(T, H, DKV).astype(np.float32)
+    scores, idx = [], np.full((T, K), -1, np.int32)
+    for t in range(T):
+        n = orc.n_avail(t, M, NC)
+        s = orc.index_scores_f32(p["qI"][t], p["w"][t], kI[:n])
+        scores.append(s)
+        idx[t] = orc.topk(s, K)
+    o = np.zeros((T, H, DV))
+    lse = np.zeros((T, H))
+    for t in range(T):
+        o[t], lse[t] = orc.csa_attend(q[t].astype(np.float64), comp.astype(np.float64), idx[t],
+                                      win.astype(np.float64), 0, t, W, DV, SCALE)
+    y = np.stack([orc.group_oproj(o[t], p["Wg"].astype(np.float64), p["Wo"].astype(np.float64)) for t in range(T)])
+    return dict(win=win, q=q, scores=scores, idx=idx, o=o, lse=lse, y=y)
+
+
+def _t(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def test_c1_chain(L, orc):
+    p = _inputs()
+    pos = torch.arange(T, dtype=torch.int64, device=DEV)
+
+    # ---- 1. compressors: KV (RoPE on the last 16 dims) and index keys
+    comp_ref, _ = orc.compress(p["x"], p["z"], p["bias"], M, OV, d_rope=DR)
+    kI_ref, _ = orc.compress(p["kx"], p["zI"], p["biasI"], M, OV, d_rope=0)
+    comp_g = L.csa_compress(_t(p["x"])[None], _t(p["z"])[None], _t(p["bias"]), m=M, overlap=OV, d_rope=DR)
+    kI_g = L.csa_compress(_t(p["kx"])[None], _t(p["zI"])[None], _t(p["biasI"]), m=M, overlap=OV, d_rope=0)
+    assert_close_abs(comp_g[0].cpu().numpy(), comp_ref, 1e-4, "compressed KV")
+    assert_close_abs(kI_g[0].cpu().numpy(), kI_ref, 1e-4, "compressed index keys")
+    comp_o = comp_ref.astype(np.float32)
+    kI_o = kI_ref.astype(np.float32)
+    ref = _oracle_chain(orc, p, comp_o, kI_o)
+
+    # ---- 2. indexer + top-k on the oracle's entries: bit-exact
+    q_pos = pos.view(1, T)
+    idx_g, sc_g = L.csa_index_topk(_t(p["qI"])[None], _t(p["w"])[None], _t(kI_o)[None], K, q_pos=q_pos, m=M,
+                                   want_scores=True)
+    idx_g, sc_g = idx_g[0].cpu().numpy(), sc_g[0].cpu().numpy()
+    for t in range(T):
+        n = orc.n_avail(t, M, NC)
+        np.testing.assert_array_equal(sc_g[t, :n], ref["scores"][t], err_msg=f"scores of query {t}")
+    np.testing.assert_array_equal(idx_g, ref["idx"])
+    assert np.all(ref["idx"][:3] == -1)               # no entry is complete before token 3
+
+    # ---- 3. attention on the oracle's entries, window rows, queries and selection
+    wp0 = torch.zeros(1, dtype=torch.int64, device=DEV)
+    o_g, lse_g = L.csa_attend(_t(ref["q"])[None], _t(comp_o)[None], _t(ref["win"])[None], _t(ref["idx"])[None], DV,
+                              SCALE, q_pos=q_pos, win_pos0=wp0, W=W, want_lse=True)
+    assert_close_abs(o_g[0].cpu().numpy(), ref["o"], 1e-4, "attention")
+    assert_close_abs(lse_g[0].cpu().numpy(), ref["lse"], 1e-4, "attention lse")
+
+    # ---- 4. grouped output projection on the oracle's attention output
+    y_g = L.group_oproj(_t(ref["o"].astype(np.float32)), _t(p["Wg"]), _t(p["Wo"]))
+    assert_close_abs(y_g.cpu().numpy(), ref["y"], 1e-4, "grouped projection")
+
+    # ---- 5. the whole chain on the GPU's own intermediates
+    win_g = L.lcs_rope(_t(p["x"]).clone(), pos, DR)
+    q_g = L.lcs_rope(_t(p["q_raw"]).clone(), pos.repeat_interleave(H), DR)
+    idx_c, sc_c = L.csa_index_topk(_t(p["qI"])[None], _t(p["w"])[None], kI_g, K, q_pos=q_pos, m=M, want_scores=True)
+    o_c = L.csa_attend(q_g[None], comp_g, win_g[None], idx_c, DV, SCALE, q_pos=q_pos, win_pos0=wp0, W=W)
+    y_c = L.group_oproj(o_c[0], _t(p["Wg"]), _t(p["Wo"])).cpu().numpy()
+    idx_c = idx_c[0].cpu().numpy()
+    # When the keys move by at most eps, a score moves by at most
+    #   sum_h |w_h| (eps sum_d |qI_hd| + (d_I+1) 2^-23 sum_d |qI_hd||k_d|) + (H_I+1) 2^-23 sum_h |w_h||dot_h|
+    # (the key change, and a rounding of each fma chain that may land differently).
+    kI_gn = kI_g[0].cpu().numpy().astype(np.float64)
+    eps = float(np.max(np.abs(kI_gn - kI_ref)))
+    ka = np.abs(kI_ref) + eps
+    near = []
+    for t in range(T):
+        n = orc.n_avail(t, M, NC)
+        if n <= K:
+            np.testing.assert_array_equal(idx_c[t], ref["idx"][t])
+        else:
+            srt = np.sort(ref["scores"][t].astype(np.float64))[::-1]
+            qa = np.abs(p["qI"][t]).astype(np.float64)
+            wa = np.abs(p["w"][t]).astype(np.float64)
+            sabs = ka[:n] @ qa.T                                              # [n, H_I]
+            per_key = (eps * qa.sum(axis=1) + (DI + 1) * 2.0 ** -23 * sabs) @ wa + (HI + 1) * 2.0 ** -23 * (sabs @ wa)
+            bound = float(per_key.max())
+            if srt[K - 1] - srt[K] <= 2 * bound:
+                near.append(t)
+                continue
+            np.testing.assert_array_equal(idx_c[t], ref["idx"][t], err_msg=f"chain selection of query {t}")
+        assert_close_abs(y_c[t], ref["y"][t], 1e-4, f"chain output of query {t}")
+    print(f"\nC1 chain: {T} queries, {len(near)} near-ties excluded from the chain comparison: {near}")
+    assert len(near) <= 8

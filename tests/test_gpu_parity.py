@@ -169,7 +169,7 @@ def test_index_bf16_tensor_cores(L, orc):
     kI = randn("g.ib.k", (B, Nc, dI), dtype=torch.bfloat16)
     idx, sc = L.csa_index_topk(qI.to(DEV), w.to(DEV), kI.to(DEV), k, want_scores=True)
     idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
-    exact_rows = 0
+    near = []
     for b in range(B):
         qd, kd, wd = qI[b, 0].double().numpy(), kI[b].double().numpy(), w[b, 0].numpy()
         ref = orc.index_scores_bf16(qd, wd, kd)
@@ -181,8 +181,43 @@ def test_index_bf16_tensor_cores(L, orc):
         # level 3: when the oracle's k-th gap exceeds twice the bound, the sets agree
         if topk_gap_ok(ref, k, bound.max()):
             np.testing.assert_array_equal(idx[b, 0], orc.topk(ref, k))
-            exact_rows += 1
-    assert exact_rows >= B // 2
+        else:
+            near.append(b)
+    print(f"\nbf16 indexer: {B} rows, near-ties {near}")
+    assert len(near) <= 1, f"near-ties {near}: more than expected from the bound"
+
+
+def test_index_bf16_dot_rounding(L, orc):
+    """How the tensor cores round a 128-long bf16 dot (kind::f16, fp32 accumulation):
+    with a one-hot head weight the score is exactly ReLU of one head's dot, which the
+    oracle defines as the exact dot rounded once to fp32.  Every GPU dot must lie within
+    the derived bound of it; the share that equals it is reported (when it is all of them,
+    bf16-key selections are bit-exact end to end)."""
+    B, H, dI, Nc = 64, 64, 128, 2048
+    qI = randn("g.ir.q", (B, 1, H, dI), dtype=torch.bfloat16)
+    kI = randn("g.ir.k", (B, Nc, dI), dtype=torch.bfloat16)
+    w = torch.zeros((B, 1, H))
+    for b in range(B):
+        w[b, 0, b % H] = 1.0                       # request b tests head b's accumulator column
+    tot = eq = 0
+    worst = 0.0
+    for sign in (1.0, -1.0):                       # the negated query turns the other half positive
+        q_s = (qI * sign).contiguous()
+        _, sc = L.csa_index_topk(q_s.to(DEV), w.to(DEV), kI.to(DEV), 1, want_scores=True)
+        sc = sc.cpu().numpy()[:, 0]
+        for b in range(B):
+            qd, kd = q_s[b, 0].double().numpy(), kI[b].double().numpy()
+            ref = orc.index_scores_bf16(qd, w[b, 0].numpy(), kd).astype(np.float64)
+            pos = ref > 0
+            g = sc[b].astype(np.float64)
+            bound = (dI // 16 + 1) * 2.0 ** -23 * (np.abs(kd) @ np.abs(qd[b % H]))
+            assert np.all(np.abs(g - ref) <= bound), f"b={b}: a dot outside the bound"
+            tot += int(pos.sum())
+            eq += int((g[pos] == ref[pos]).sum())
+            worst = max(worst, float(np.max(np.abs(g - ref)[pos] / bound[pos])))
+    print(f"\nkind::f16 128-dot: {eq}/{tot} equal to the correctly rounded dot "
+          f"({100.0 * eq / tot:.2f} %), largest error {worst:.3f} of the bound")
+    assert tot > B * Nc // 2
 
 
 @pytest.mark.parametrize("B,Q", [(1, 40), (2, 38)])   # 38: the last group of four queries is ragged
@@ -490,14 +525,28 @@ def test_decode_fused_csa_bf16(L, orc):
                                                  qI=qI.to(DEV), w=w.to(DEV), kI=kI.to(DEV), k=k, idx_out=idx_out,
                                                  out_dtype=od))
     out, idx = out.cpu().numpy(), idx_out.cpu().numpy()
+    near = []
+    ref_idx = np.zeros((B, k), np.int32)
     for b in range(B):
         qd, kd, wd = qI[b].double().numpy(), kI[b].double().numpy(), w[b].numpy()
         ref_s = orc.index_scores_bf16(qd, wd, kd)
+        ref_idx[b] = orc.topk(ref_s, k)
         if topk_gap_ok(ref_s, k, _bf16_score_bound(qd, wd, kd).max()):
-            np.testing.assert_array_equal(idx[b], orc.topk(ref_s, k))
-        o, _ = orc.csa_attend(q[b].double().numpy(), comp[b].double().numpy(), idx[b], win[b].double().numpy(), 0,
-                              -1, 128, dv, scale)
-        assert_close_rel_rms(out[b], o, 2e-2, f"fused b {b}")
+            np.testing.assert_array_equal(idx[b], ref_idx[b])
+        else:
+            near.append(b)
+    assert len(near) <= 1, f"near-ties {near}"
+    # attention on the oracle's selection: the fused step's output where the selections
+    # agree, else csa_attend given the oracle's selection
+    att = both_outputs(lambda od: L.csa_attend(q.to(DEV).view(B, 1, H, D), comp.to(DEV), win.to(DEV),
+                                               torch.from_numpy(ref_idx).to(DEV).view(B, 1, k), dv, scale,
+                                               out_dtype=od)).cpu().numpy()[:, 0]
+    for b in range(B):
+        if b not in near:
+            np.testing.assert_array_equal(out[b], att[b])
+        o, _ = orc.csa_attend(q[b].double().numpy(), comp[b].double().numpy(), ref_idx[b],
+                              win[b].double().numpy(), 0, -1, 128, dv, scale)
+        assert_close_rel_rms(att[b], o, 2e-2, f"fused b {b}")
 
 
 def test_decode_fused_hca(L, orc):

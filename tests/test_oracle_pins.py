@@ -217,6 +217,30 @@ def test_compress_one_hot_selects_the_token(orc):
                 np.testing.assert_array_equal(e[j], x[t])
 
 
+def test_compress_one_hot_logit_selects_its_token(orc):
+    """The pooling logit of token t weights token t ("DeepSeek V4 深度解析" §2, CSA step 1:
+    one learned weight per raw token).  With zero bias and one token's logit far above the
+    rest, every entry whose window holds that token is exactly that token's row, and every
+    other entry is the plain mean of its window.  Reading the logit of a neighbouring token
+    (either direction) or a window shifted by one fails here."""
+    T, d = 64, 8
+    x = synth.normal("pin.c.zoh", (T, d))
+    for m, ov in ((4, 2), (4, 0), (8, 3)):
+        W = m + ov
+        for hot in (0, 1, 5, 6, 30, 33, T - 1):
+            z = np.zeros(T)
+            z[hot] = 1e4                       # exp(-1e4) underflows to 0 in double
+            e, pw = orc.compress(x, z, np.zeros(W), m=m, overlap=ov)
+            for j in range(T // m):
+                lo = m * j - ov
+                ts = [t for t in range(lo, lo + W) if 0 <= t < T]
+                if hot in ts:
+                    np.testing.assert_array_equal(e[j], x[hot], err_msg=f"m={m} ov={ov} hot={hot} j={j}")
+                    assert pw[j, hot - lo] == 1.0
+                else:
+                    np.testing.assert_allclose(e[j], x[ts].mean(axis=0), rtol=0, atol=1e-14)
+
+
 def test_compress_weights_sum_to_one_and_mean(orc):
     x = synth.normal("pin.c.s", (256, 16))
     z = 3 * synth.normal("pin.c.sz", 256)
