@@ -134,7 +134,9 @@ LCS_API int hca_compress(const void* x, int x_dtype, int64_t B, int64_t T, int d
  *   scores [B, Q, N_c] score_dtype, optional output (NULL: kept in the workspace);
  *                         entries s >= n_avail are unspecified
  * score_dtype: LCS_F32 (kI F32 or BF16) or LCS_BF16 (kI FP4).  d_I % 32 == 0,
- * H_I <= 128 (LCS_F32 path) or H_I == 64 (tensor-core paths).
+ * H_I <= 128 (LCS_F32 path) or H_I == 64 (tensor-core paths).  Tensor-core paths:
+ * qI and kI start on a 16-byte boundary, an LCS_FP4 kI on a 32-byte boundary
+ * (else LCS_ERR_INVALID).
  */
 LCS_API int csa_index_topk(const void* qI, int qI_dtype, const float* w, const void* kI, int kI_dtype,
                    int64_t B, int64_t Q, int64_t N_c, int H_I, int d_I,
@@ -248,6 +250,42 @@ LCS_API int decode_fused(int mode, int64_t B,
                  int H_I, int d_I, int k, int score_dtype,
                  void* out, int out_dtype, float* lse, int32_t* idx_out,
                  void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Decode-time cache update ("DeepSeek V4 深度解析" §4, KV-cache management for the
+ * mixed attention: a state cache holding the sliding window and the raw tokens not yet
+ * enough to compress, and a compressed cache of CSA and HCA entries).  Appends one new
+ * token to each request; request b's token sits at position t = pos[b] (the number of
+ * tokens the request had before), and pos[b] < 0 appends nothing to request b.
+ *   state cache:  raw    [B, 128, D + d_I] x_dtype  ring of the last 128 raw (un-rotated)
+ *                        tokens, KV row then index-key row, slot t % 128;
+ *                 logits [B, 3, 128] fp32  ring of the tokens' pooling logits (z, zI, zh);
+ *                 win    [B, 128, row] win_dtype  the window: slot t % 128 receives the
+ *                        token's KV row rotated at position t (the rows csa_attend reads);
+ *   compressed cache, written when an entry's last token arrives:
+ *                 comp [B, N_c, row] kv_dtype   CSA entry j = t/4 when (t+1) % 4 == 0: tokens
+ *                        4j-2 .. 4j+3 (those >= 0) pooled with softmax(z + bias[0..5]), then
+ *                        rotated at position t (as csa_compress with m = 4, overlap 2);
+ *                 kI   [B, N_c, d_I] or FP4 planes (kI_dtype)  index key j, pooled the same
+ *                        way from the index-key rows with zI and biasI, no rotation;
+ *                 hca  [B, N_h, row] kv_dtype   HCA entry h = t/128 when (t+1) % 128 == 0:
+ *                        tokens 128h .. 128h+127 pooled with softmax(zh + biash[0..127]),
+ *                        rotated at position t (as hca_compress with m' = 128).
+ *   x [B, D], kx [B, d_I]  x_dtype (LCS_F32 or LCS_BF16) the new token's raw rows;
+ *   z, zI, zh [B] fp32; bias [6], biasI [6], biash [128] fp32.
+ * Storage: kv_dtype and win_dtype LCS_F32, LCS_BF16 or LCS_KV_FP8 (content D - d_rope a
+ * multiple of 128; quantised exactly as lcs_quant_kv_fp8 quantises the fp32 entry);
+ * kI_dtype LCS_F32, LCS_BF16 or LCS_FP4 (as lcs_quant_fp4).  The rings are read only at
+ * slots of tokens already appended.  An entry index >= N_c or >= N_h is not written and
+ * records LCS_ERR_DEVICE in the status word of ws (>= 256 bytes, 256-byte aligned).
+ * D % 8 == 0, d_I % 32 == 0, d_rope even.
+ */
+LCS_API int lcs_cache_append(int64_t B, const int64_t* pos, const void* x, const void* kx, int x_dtype,
+                 const float* z, const float* zI, const float* zh,
+                 const float* bias, const float* biasI, const float* biash,
+                 int D, int d_rope, int d_I, float rope_theta, void* raw, float* logits,
+                 void* win, int win_dtype, void* comp, void* kI, void* hca, int64_t N_c, int64_t N_h,
+                 int kv_dtype, int kI_dtype, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
  * Grouped output projection ("DeepSeek V4 深度解析" §2, HCA paragraph: both use a

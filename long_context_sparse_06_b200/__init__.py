@@ -15,7 +15,7 @@ import os
 __all__ = [
     "F32", "BF16", "KV_FP8", "FP4", "MODE_CSA", "MODE_HCA", "LcsError", "lib",
     "csa_compress", "hca_compress", "csa_index_topk", "lcs_topk", "csa_attend", "hca_attend",
-    "decode_fused", "group_oproj", "lcs_rope", "lcs_quant_kv_fp8", "lcs_quant_fp4",
+    "decode_fused", "lcs_cache_append", "group_oproj", "lcs_rope", "lcs_quant_kv_fp8", "lcs_quant_fp4",
     "lcs_workspace_size", "lcs_status", "lcs_clear_status", "lcs_selftest_wait", "workspace", "kv_fp8_row_bytes",
 ]
 
@@ -54,6 +54,8 @@ def lib():
             "csa_attend": [P, I, P, P, I, I64, I64, I64, I64, P, I, P, P, I, I, I, I, F, P, I, P, P, SZ, P],
             "csa_attend_noalloc": [P, I, P, P, I, I64, I64, I64, I64, P, I, P, P, I, I, I, I, F, P, I, P, P, P],
             "hca_attend": [P, I, P, P, I, I64, I64, I64, I64, P, P, I, I, I, I, I, F, P, I, P, P, SZ, P],
+            "lcs_cache_append": [I64, P, P, P, I, P, P, P, P, P, P, I, I, I, F, P, P, P, I, P, P, P, I64, I64, I, I,
+                                 P, SZ, P],
             "decode_fused": [I, I64, P, I, P, P, I, I64, I64, I, I, I, F, P, I, P, P, I, I, I, I, I, P, I, P, P, P,
                              SZ, P],
             "group_oproj": [P, I64, I, I, P, I, I, P, I, P, P],
@@ -293,6 +295,34 @@ def decode_fused(mode, q, comp, win, d_v, scale, kv_dtype=None, qI=None, w=None,
           _ptr(qI), qI_dt, _ptr(w), _ptr(kI), kI_dtype, H_I, d_I, k, score_dtype, _ptr(out), _dt(out), _ptr(lse),
           _ptr(idx_out), _ptr(ws), ws.numel(), _stream(stream))
     return (out, lse) if want_lse else out
+
+
+# ------------------------------------------------------- decode cache update
+def lcs_cache_append(pos, x, kx, z, zI, zh, bias, biasI, biash, raw, logits, win, comp, kI, hca, d_rope=64,
+                     rope_theta=10000.0, win_dtype=None, kv_dtype=None, kI_dtype=None, N_c=None, ws=None,
+                     stream=None):
+    """Appends one token per request (pos [B] int64; negative: no token for that request).
+    x [B,D], kx [B,d_I] (fp32/bf16); z, zI, zh [B]; rings raw [B,128,D+d_I], logits
+    [B,3,128]; caches win [B,128,row], comp [B,N_c,row], kI [B,N_c,d_I] or FP4 planes,
+    hca [B,N_h,row].  The storage dtypes default to the tensors' own (uint8 rows: FP8 KV)."""
+    B, D = x.shape
+    d_I = kx.shape[1]
+    u8 = _torch().uint8
+    if kv_dtype is None:
+        kv_dtype = KV_FP8 if comp.dtype == u8 else _dt(comp)
+    if win_dtype is None:
+        win_dtype = KV_FP8 if win.dtype == u8 else _dt(win)
+    if kI_dtype is None:
+        kI_dtype = FP4 if kI.dtype == u8 else _dt(kI)
+    if N_c is None:
+        N_c = comp.shape[1]
+    if ws is None:
+        ws = workspace(256, x.device)
+    _call("lcs_cache_append", B, _ptr(pos), _ptr(x), _ptr(kx), _dt(x), _ptr(z), _ptr(zI), _ptr(zh), _ptr(bias),
+          _ptr(biasI), _ptr(biash), D, d_rope, d_I, rope_theta, _ptr(raw), _ptr(logits), _ptr(win), win_dtype,
+          _ptr(comp), _ptr(kI), _ptr(hca), N_c, hca.shape[1], kv_dtype, kI_dtype, _ptr(ws), ws.numel(),
+          _stream(stream))
+    return ws
 
 
 # --------------------------------------------------------------------- misc

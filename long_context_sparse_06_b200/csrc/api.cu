@@ -278,7 +278,8 @@ static int validate_index(const void* qI, int qI_dtype, const float* w, const vo
     }
     if (qI_dtype == LCS_BF16 && kI_dtype == LCS_FP4) {
         if (score_dtype != LCS_BF16 || H_I != 64 || d_I != 128) return LCS_ERR_UNSUPPORTED;
-        if (!aligned16(qI) || !aligned16(kI)) return LCS_ERR_INVALID;
+        // the packed key plane is read by TMA in the 16-byte-slot FP4 form, which needs 32 bytes
+        if (!aligned16(qI) || (reinterpret_cast<uintptr_t>(kI) & 31)) return LCS_ERR_INVALID;
         return LCS_OK;
     }
     return LCS_ERR_UNSUPPORTED;
@@ -471,6 +472,34 @@ int decode_fused(int mode, int64_t B, const void* q, int q_dtype, const void* co
         return LCS_ERR_CUDA;
     record_stage(csa ? 3 : 1, stream);
     return LCS_OK;
+}
+
+// ------------------------------------------------------- decode cache update
+int lcs_cache_append(int64_t B, const int64_t* pos, const void* x, const void* kx, int x_dtype, const float* z,
+                     const float* zI, const float* zh, const float* bias, const float* biasI, const float* biash,
+                     int D, int d_rope, int d_I, float rope_theta, void* raw, float* logits, void* win, int win_dtype,
+                     void* comp, void* kI, void* hca, int64_t N_c, int64_t N_h, int kv_dtype, int kI_dtype, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+    if (pos == nullptr || x == nullptr || kx == nullptr || z == nullptr || zI == nullptr || zh == nullptr ||
+        bias == nullptr || biasI == nullptr || biash == nullptr || raw == nullptr || logits == nullptr ||
+        win == nullptr || comp == nullptr || kI == nullptr || hca == nullptr)
+        return LCS_ERR_INVALID;
+    if (B < 0 || N_c < 0 || N_h < 0 || D <= 0 || D > 4096 || D % 8 || d_I <= 0 || d_I > 1024 || d_I % 32 ||
+        d_rope < 0 || d_rope > D || (d_rope & 1) || !(rope_theta > 0.f))
+        return LCS_ERR_INVALID;
+    if (x_dtype != LCS_F32 && x_dtype != LCS_BF16) return LCS_ERR_UNSUPPORTED;
+    const bool kv_ok = kv_dtype == LCS_F32 || kv_dtype == LCS_BF16 || (kv_dtype == LCS_KV_FP8 && (D - d_rope) % 128 == 0);
+    const bool win_ok = win_dtype == LCS_F32 || win_dtype == LCS_BF16 || (win_dtype == LCS_KV_FP8 && (D - d_rope) % 128 == 0);
+    if (!kv_ok || !win_ok || (kI_dtype != LCS_F32 && kI_dtype != LCS_BF16 && kI_dtype != LCS_FP4))
+        return LCS_ERR_UNSUPPORTED;
+    if ((kv_dtype == LCS_KV_FP8 || win_dtype == LCS_KV_FP8) && (!aligned16(comp) || !aligned16(win) || !aligned16(hca)))
+        return LCS_ERR_INVALID;
+    if (ws == nullptr || ws_bytes < (size_t)kStatusBytes || (reinterpret_cast<uintptr_t>(ws) & 255))
+        return LCS_ERR_WORKSPACE;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    return from_cuda(launch_cache_append(pos, x, kx, x_dtype, z, zI, zh, bias, biasI, biash, D, d_rope, d_I,
+                                         rope_theta, raw, logits, win, win_dtype, comp, kI, hca, B, N_c, N_h, kv_dtype,
+                                         kI_dtype, status_of(ws), stream));
 }
 
 // ------------------------------------------------------------------- misc

@@ -380,6 +380,63 @@ __device__ __forceinline__ uint32_t bf16_key(uint16_t b) {
     return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
 }
 
+// ------------------------------------------------------ shared cache writers
+// Rotate-half RoPE of one pair (x1 at dim c0 + i, x2 at dim c0 + i + d_rope/2) at position
+// pos: angle pos * theta^(-2i/d_rope), formed and reduced in double so that positions near
+// 2^20 keep full fp32 accuracy after the reduction.
+__device__ __forceinline__ void rope_pair(float x1, float x2, int64_t pos, int i, int d_rope, float theta, float& o1,
+                                          float& o2) {
+    const double freq = pow((double)theta, -2.0 * i / (double)d_rope);
+    double a = (double)pos * freq;
+    a -= 6.283185307179586 * rint(a * 0.15915494309189535);
+    float sn, cs;
+    sincosf((float)a, &sn, &cs);
+    o1 = x1 * cs - x2 * sn;
+    o2 = x2 * cs + x1 * sn;
+}
+
+__device__ __forceinline__ float warp_max(float v);
+
+// One warp writes one mixed-precision KV row: each 128-dim content block as E4M3 codes of
+// x / scale with the smallest power-of-two scale >= amax/448 (1 when amax is 0), then the
+// d_r RoPE dims as bf16, then the fp32 scales.  xr: d_c + d_r floats, 16-byte aligned.
+__device__ __forceinline__ void quant_kv_fp8_row_warp(const float* xr, int d_c, int d_r, uint8_t* o) {
+    const int lane = threadIdx.x & 31;
+    const int nb = d_c / 128;
+    for (int b = 0; b < nb; ++b) {
+        const float4 v = *reinterpret_cast<const float4*>(xr + b * 128 + 4 * lane);
+        float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+        amax = warp_max(amax);
+        // smallest power of two >= amax/448: round the fp32 bit pattern up to the next exponent
+        const float t = amax / 448.0f;
+        const uint32_t tb = __float_as_uint(t);
+        const float sc = (t > 0.0f) ? __uint_as_float((tb + 0x007FFFFFu) & 0xFF800000u) : 1.0f;
+        const uint32_t c = (uint32_t)f32_to_e4m3(v.x / sc) | ((uint32_t)f32_to_e4m3(v.y / sc) << 8) |
+                           ((uint32_t)f32_to_e4m3(v.z / sc) << 16) | ((uint32_t)f32_to_e4m3(v.w / sc) << 24);
+        *reinterpret_cast<uint32_t*>(o + b * 128 + 4 * lane) = c;
+        if (lane == 0) *reinterpret_cast<float*>(o + d_c + 2 * d_r + 4 * b) = sc;
+    }
+    for (int j = lane; j < d_r; j += 32) {
+        const uint16_t h = f32_to_bf16_bits(xr[d_c + j]);
+        *reinterpret_cast<uint16_t*>(o + d_c + 2 * j) = h;
+    }
+}
+
+// One warp quantises one 32-element FP4 block (lane = element v): scale = E4M3(amax/6), 1
+// when that is 0; code = E2M1(v / scale).  Writes the 16 packed bytes (element 2j in the
+// low nibble of byte j) and the scale byte.
+__device__ __forceinline__ void quant_fp4_block_warp(float v, uint8_t* packed16, uint8_t* scale) {
+    const int lane = threadIdx.x & 31;
+    const float amax = warp_max(fabsf(v));
+    uint8_t sc_code = f32_to_e4m3(amax / 6.0f);
+    if ((sc_code & 0x7F) == 0) sc_code = 0x38;   // 1.0
+    const float sc = e4m3_to_f32(sc_code);
+    const uint32_t q = f32_to_e2m1(v / sc);
+    const uint32_t other = __shfl_down_sync(0xffffffffu, q, 1);
+    if ((lane & 1) == 0) packed16[lane / 2] = (uint8_t)(q | (other << 4));
+    if (lane == 0) *scale = sc_code;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

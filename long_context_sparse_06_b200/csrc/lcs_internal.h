@@ -69,6 +69,13 @@ struct AttendArgs {
 int64_t attend_scratch_bytes(const AttendArgs& a);
 cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaStream_t s, bool pdl);
 
+// cache.cu -- decode-time cache update (one token per request)
+cudaError_t launch_cache_append(const int64_t* pos, const void* x, const void* kx, int x_dtype, const float* z,
+                                const float* zI, const float* zh, const float* bias, const float* biasI,
+                                const float* biash, int D, int d_rope, int d_I, float theta, void* raw,
+                                float* logits, void* win, int win_dtype, void* comp, void* kI, void* hca, int64_t B,
+                                int64_t N_c, int64_t N_h, int kv_dtype, int kI_dtype, int* status, cudaStream_t s);
+
 // noalloc.cu -- device address of the fixed scratch array behind csa_attend_noalloc
 // for the current device (looked up once per device).  LCS_OK or LCS_ERR_CUDA.
 int noalloc_scratch(void** ptr);

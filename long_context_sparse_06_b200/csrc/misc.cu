@@ -18,8 +18,7 @@ namespace lcs {
 
 namespace {
 
-// One thread per (row, pair).  The angle is formed and reduced in double so that
-// positions near 2^20 keep full fp32 accuracy after the reduction.
+// One thread per (row, pair).
 template <typename T>
 __global__ void rope_kernel(T* rows, int64_t n, int d, int d_rope, float theta, const int64_t* __restrict__ pos) {
     const int half = d_rope / 2;
@@ -28,67 +27,34 @@ __global__ void rope_kernel(T* rows, int64_t n, int d, int d_rope, float theta, 
     const int64_t r = g / half;
     const int i = (int)(g - r * half);
     const int c0 = d - d_rope;
-    const double freq = pow((double)theta, -2.0 * i / (double)d_rope);
-    double a = (double)pos[r] * freq;
-    a -= 6.283185307179586 * rint(a * 0.15915494309189535);
-    float sn, cs;
-    sincosf((float)a, &sn, &cs);
     T* x = rows + r * d;
+    float o1, o2;
     if constexpr (sizeof(T) == 4) {
-        const float x1 = x[c0 + i], x2 = x[c0 + i + half];
-        x[c0 + i] = x1 * cs - x2 * sn;
-        x[c0 + i + half] = x2 * cs + x1 * sn;
+        rope_pair(x[c0 + i], x[c0 + i + half], pos[r], i, d_rope, theta, o1, o2);
+        x[c0 + i] = o1;
+        x[c0 + i + half] = o2;
     } else {
-        const float x1 = __bfloat162float(x[c0 + i]), x2 = __bfloat162float(x[c0 + i + half]);
-        x[c0 + i] = __float2bfloat16_rn(x1 * cs - x2 * sn);
-        x[c0 + i + half] = __float2bfloat16_rn(x2 * cs + x1 * sn);
+        rope_pair(__bfloat162float(x[c0 + i]), __bfloat162float(x[c0 + i + half]), pos[r], i, d_rope, theta, o1, o2);
+        x[c0 + i] = __float2bfloat16_rn(o1);
+        x[c0 + i + half] = __float2bfloat16_rn(o2);
     }
 }
 
 // One warp per row.  Each 128-dim block: lane l owns elements 4l..4l+3.
 __global__ void quant_kv_fp8_kernel(const float* __restrict__ x, int64_t n, int d_c, int d_r,
                                     uint8_t* __restrict__ out) {
-    const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= n) return;
-    const int nb = d_c / 128;
-    const int64_t rb = d_c + 2 * d_r + 4 * nb;
-    const float* xr = x + r * (d_c + d_r);
-    uint8_t* o = out + r * rb;
-    for (int b = 0; b < nb; ++b) {
-        const float4 v = *reinterpret_cast<const float4*>(xr + b * 128 + 4 * lane);
-        float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-        amax = warp_max(amax);
-        // smallest power of two >= amax/448: round the fp32 bit pattern up to the next exponent
-        const float t = amax / 448.0f;
-        const uint32_t tb = __float_as_uint(t);
-        const float sc = (t > 0.0f) ? __uint_as_float((tb + 0x007FFFFFu) & 0xFF800000u) : 1.0f;
-        const uint32_t c = (uint32_t)f32_to_e4m3(v.x / sc) | ((uint32_t)f32_to_e4m3(v.y / sc) << 8) |
-                           ((uint32_t)f32_to_e4m3(v.z / sc) << 16) | ((uint32_t)f32_to_e4m3(v.w / sc) << 24);
-        *reinterpret_cast<uint32_t*>(o + b * 128 + 4 * lane) = c;
-        if (lane == 0) *reinterpret_cast<float*>(o + d_c + 2 * d_r + 4 * b) = sc;
-    }
-    for (int j = lane; j < d_r; j += 32) {
-        const uint16_t h = f32_to_bf16_bits(xr[d_c + j]);
-        *reinterpret_cast<uint16_t*>(o + d_c + 2 * j) = h;
-    }
+    const int64_t rb = d_c + 2 * d_r + 4 * (d_c / 128);
+    quant_kv_fp8_row_warp(x + r * (d_c + d_r), d_c, d_r, out + r * rb);
 }
 
 // One warp per 32-element block, lane = element.
 __global__ void quant_fp4_kernel(const float* __restrict__ x, int64_t nblk, uint8_t* __restrict__ packed,
                                  uint8_t* __restrict__ scales) {
-    const int lane = threadIdx.x & 31;
     const int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (blk >= nblk) return;
-    const float v = x[blk * 32 + lane];
-    const float amax = warp_max(fabsf(v));
-    uint8_t sc_code = f32_to_e4m3(amax / 6.0f);
-    if ((sc_code & 0x7F) == 0) sc_code = 0x38;   // 1.0
-    const float sc = e4m3_to_f32(sc_code);
-    const uint32_t q = f32_to_e2m1(v / sc);
-    const uint32_t other = __shfl_down_sync(0xffffffffu, q, 1);
-    if ((lane & 1) == 0) packed[blk * 16 + lane / 2] = (uint8_t)(q | (other << 4));
-    if (lane == 0) scales[blk] = sc_code;
+    quant_fp4_block_warp(x[blk * 32 + (threadIdx.x & 31)], packed + blk * 16, scales + blk);
 }
 
 // One block per token: the group projections into shared memory, then Wo.

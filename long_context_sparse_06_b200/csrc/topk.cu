@@ -10,7 +10,10 @@
 // element is ranked by the 64-bit composite (key << 32 | ~index), so "larger
 // composite" is exactly "larger score, then lower index".
 //
-// One CTA of 512 threads per query row:
+// Rows of at most 32768 entries (decode over 128K tokens, the tiny prefill): one CTA of
+// 1024 threads per row with the whole row in registers and an exact radix select
+// (topk_row_kernel, below).  Longer rows: one CTA of 512 threads per query row, or a
+// cluster of them per row when there are few rows:
 //  1. Lower bound: a fixed strided sample of 512 keys is histogrammed over the
 //     top 14 key bits (sign, exponent, top mantissa bits); the lower edge of the
 //     bin holding the sample's rank-r element, r about 1.5 k x sample/row + 8,
@@ -491,6 +494,218 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
     }
 }
 
+// ------------------------------------------------------ rows held in registers
+// Rows of at most kRowT * kRowKPT entries: one CTA of kRowT threads per row, thread t
+// holding the kRowKPT consecutive keys starting at t * kRowKPT (so thread order is index
+// order), in registers and mirrored in shared memory for the passes that visit only a
+// thread's remaining candidates (a 32-bit mask per thread).  An exact MSB-first radix select finds the k-th largest key:
+// each pass histograms the next digit of the keys that still share the resolved prefix,
+// and a block scan from the top bin finds the digit holding the k-th; the select stops
+// early once the remaining count equals that bin's population (the whole bin is taken).
+// One more block scan then places every selected key: all keys above the threshold, and
+// the lowest-index ones equal to it, in ascending index order.
+constexpr int kRowT = 1024, kRowKPT = 32, kRowBins = 2048;
+
+template <bool BF16>
+__global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restrict__ scores, int64_t N_c,
+                                                            const int64_t* __restrict__ q_pos, int m, int k,
+                                                            int32_t* __restrict__ idx_out) {
+    extern __shared__ uint32_t ks[];   // [kRowKPT][kRowT]: key j of thread t at ks[j * kRowT + t]
+    __shared__ uint32_t hist[kRowBins];
+    __shared__ uint32_t wsum[2][32];
+    __shared__ uint32_t s_digit, s_above, s_inbin;
+    constexpr int kBits = BF16 ? 16 : 32;
+    const int64_t row = blockIdx.x;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    int64_t n = N_c;
+    if (q_pos != nullptr) {
+        const int64_t a = (q_pos[row] + 1) / m;
+        n = a < N_c ? (a < 0 ? 0 : a) : N_c;
+    }
+    int32_t* out = idx_out + row * k;
+    const char* srow = static_cast<const char*>(scores) + row * N_c * (BF16 ? 2 : 4);
+
+#if defined(__CUDA_ARCH__)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+
+    if (n <= k) {
+        for (int i = t; i < k; i += kRowT) out[i] = (i < n) ? i : -1;
+        return;
+    }
+
+    // ---- keys of this thread (entries at or beyond n read as key 0, below every finite score)
+    const int64_t base = (int64_t)t * kRowKPT;
+    uint32_t key[kRowKPT];
+    const bool vec = (reinterpret_cast<uintptr_t>(srow) & 15) == 0 && base + kRowKPT <= n;
+    if (vec) {
+        const uint4* p = reinterpret_cast<const uint4*>(srow + base * (BF16 ? 2 : 4));
+        constexpr int kV = kRowKPT / (BF16 ? 8 : 4);
+        uint4 raw[kV];
+#pragma unroll
+        for (int v = 0; v < kV; ++v) raw[v] = __ldg(p + v);
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            const uint32_t ww[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if constexpr (BF16) {
+                    key[v * 8 + 2 * q] = bf16_key((uint16_t)(ww[q] & 0xFFFF));
+                    key[v * 8 + 2 * q + 1] = bf16_key((uint16_t)(ww[q] >> 16));
+                } else {
+                    key[v * 4 + q] = f32_key(__uint_as_float(ww[q]));
+                }
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kRowKPT; ++j) key[j] = (base + j < n) ? load_key<BF16>(srow, base + j) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < kRowKPT; ++j) ks[j * kRowT + t] = key[j];
+
+    // ---- radix select: digits of 11, 11, 10 bits (fp32 keys) or 11, 5 (bf16 keys).  After
+    // each pass the thread keeps a mask of its keys that still share the resolved prefix, so
+    // later passes and the placement visit only those.
+    uint32_t prefix = 0, krem = (uint32_t)k;
+    uint32_t cand = 0xFFFFFFFFu;   // keys still sharing the prefix (all of them before pass 0)
+    uint32_t above = 0;            // keys already known to lie above the threshold
+    int done = 0;
+    bool whole_bin = false;
+#pragma unroll 1
+    for (int pass = 0; pass < 3 && done < kBits; ++pass) {
+        const int width = (kBits - done) < 11 ? (kBits - done) : 11;
+        const int shift = kBits - done - width;
+        const int nb = 1 << width;
+        for (int i = t; i < nb; i += kRowT) hist[i] = 0;
+        __syncthreads();
+        if (pass == 0) {
+#pragma unroll
+            for (int j = 0; j < kRowKPT; ++j) atomicAdd(&hist[key[j] >> shift], 1u);
+        } else {
+            for (uint32_t m = cand; m != 0; m &= m - 1) {
+                const uint32_t kk = ks[(__ffs(m) - 1) * kRowT + t];
+                atomicAdd(&hist[(kk >> shift) & (nb - 1)], 1u);
+            }
+        }
+        __syncthreads();
+        // bins from the top: thread t owns bins nb-1-2t and nb-2-2t (nb = 2048), or nb-1-t
+        const int per = nb >= 2 * kRowT ? 2 : 1;
+        const int b0 = nb - 1 - t * per;
+        uint32_t c0 = 0, c1 = 0;
+        if (b0 >= 0) c0 = hist[b0];
+        if (per == 2 && b0 >= 1) c1 = hist[b0 - 1];
+        const uint32_t local = c0 + c1;
+        uint32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[0][warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t v = wsum[0][lane];
+            uint32_t x = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            wsum[1][lane] = x - v;
+        }
+        __syncthreads();
+        const uint32_t excl = wsum[1][warp] + incl - local;
+        if (excl < krem && excl + local >= krem) {
+            if (excl + c0 >= krem) {
+                s_digit = (uint32_t)b0;
+                s_above = excl;
+                s_inbin = c0;
+            } else {
+                s_digit = (uint32_t)(b0 - 1);
+                s_above = excl + c0;
+                s_inbin = c1;
+            }
+        }
+        __syncthreads();
+        const uint32_t dg = s_digit;
+        prefix = (prefix << width) | dg;
+        done += width;
+        krem -= s_above;
+        // split this thread's candidates: digit above the threshold digit, or equal to it
+        uint32_t nc = 0;
+        if (pass == 0) {
+#pragma unroll
+            for (int j = 0; j < kRowKPT; ++j) {
+                const uint32_t d = key[j] >> shift;
+                above |= (d > dg ? 1u : 0u) << j;
+                nc |= (d == dg ? 1u : 0u) << j;
+            }
+        } else {
+            for (uint32_t m = cand; m != 0; m &= m - 1) {
+                const int j = __ffs(m) - 1;
+                const uint32_t d = (ks[j * kRowT + t] >> shift) & (nb - 1);
+                if (d > dg) above |= 1u << j;
+                else if (d == dg) nc |= 1u << j;
+            }
+        }
+        cand = nc;
+        if (s_inbin == krem) {   // the whole threshold bin is taken
+            whole_bin = true;
+            break;
+        }
+    }
+
+    // ---- ordered placement: keys above the threshold, then ties at it by index
+    const uint32_t gt = __popc(above), eq = __popc(cand);
+    uint32_t ig = gt, ie = eq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t yg = __shfl_up_sync(0xffffffffu, ig, o);
+        const uint32_t ye = __shfl_up_sync(0xffffffffu, ie, o);
+        if (lane >= o) {
+            ig += yg;
+            ie += ye;
+        }
+    }
+    __syncthreads();   // wsum is reused
+    if (lane == 31) {
+        wsum[0][warp] = ig;
+        wsum[1][warp] = ie;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t vg = wsum[0][lane], ve = wsum[1][lane];
+        uint32_t xg = vg, xe = ve;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t yg = __shfl_up_sync(0xffffffffu, xg, o);
+            const uint32_t ye = __shfl_up_sync(0xffffffffu, xe, o);
+            if (lane >= o) {
+                xg += yg;
+                xe += ye;
+            }
+        }
+        __syncwarp();
+        wsum[0][lane] = xg - vg;
+        wsum[1][lane] = xe - ve;
+    }
+    __syncthreads();
+    const uint32_t gt_before = wsum[0][warp] + ig - gt;
+    const uint32_t e0 = wsum[1][warp] + ie - eq;          // ties before this thread's keys
+    uint32_t take = above;
+    if (whole_bin) {
+        take |= cand;
+    } else if (e0 < krem) {   // the first krem - e0 ties of this thread
+        uint32_t m = cand;
+        for (uint32_t r = e0; r < krem && m != 0; ++r) m &= m - 1;
+        take |= cand & ~m;
+    }
+    uint32_t pos = gt_before + (whole_bin ? e0 : (e0 < krem ? e0 : krem));
+    for (uint32_t m = take; m != 0; m &= m - 1) out[pos++] = (int32_t)(base + __ffs(m) - 1);
+}
+
 }  // namespace
 
 int64_t topk_scratch_bytes(int64_t rows, int64_t N_c) {
@@ -540,6 +755,13 @@ int choose_ranks(int64_t rows, int64_t N_c) {
 template <bool BF16>
 cudaError_t launch_topk_t(const void* scores, int64_t rows, int64_t N_c, const int64_t* q_pos, int m, int k,
                           int32_t* idx, cudaStream_t s, bool pdl) {
+    if (N_c <= (int64_t)kRowT * kRowKPT) {   // the whole row fits one CTA's registers
+        constexpr size_t smem = sizeof(uint32_t) * kRowT * kRowKPT;
+        cudaError_t e = set_smem_once(reinterpret_cast<const void*>(topk_row_kernel<BF16>), smem);
+        if (e != cudaSuccess) return e;
+        return launch_k(topk_row_kernel<BF16>, dim3((unsigned)rows), dim3(kRowT), smem, s, pdl, scores, N_c, q_pos, m,
+                        k, idx);
+    }
     const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16>);
     cudaError_t e = set_smem_once(kern, sizeof(TopkSmem));
     if (e != cudaSuccess) return e;

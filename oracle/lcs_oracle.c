@@ -464,7 +464,8 @@ ORC_API void orc_index_scores_fp4(const uint8_t* q_packed, const uint8_t* q_scal
 /* The k largest of score[0..n) by (score descending, index ascending), then */
 /* returned in ascending index order, padded with -1 up to k.  -0 == +0.     */
 /* ------------------------------------------------------------------------ */
-static const float* g_sort_scores;
+/* One per thread: callers may run the oracle on several threads at once. */
+static _Thread_local const float* g_sort_scores;
 static int cmp_desc(const void* pa, const void* pb)
 {
     int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;

@@ -41,13 +41,26 @@ def oracle_pool(fn, items):
         return list(ex.map(fn, items))
 
 
-def topk_gap_ok(oracle_scores, k, bound):
-    """True when the oracle's k-th and (k+1)-th best scores differ by more than 2*bound
-    (the selection is then decided by the scores, not by rounding)."""
-    s = np.sort(np.asarray(oracle_scores, np.float64))[::-1]
-    if s.size <= k:
-        return True
-    return (s[k - 1] - s[k]) > 2 * bound
+def selection_against_oracle(orc, s_gpu, idx, ref, bound, k, what):
+    """Level 3 of the selection rule for scores the tensor cores computed: every GPU score
+    lies within `bound` of the oracle's; when the GPU selection differs from the oracle's,
+    the oracle's k-th and (k+1)-th scores must lie within twice the largest actual score
+    difference (a near-tie), and the GPU selection must still be a top-k of the oracle's
+    scores up to that difference.  Returns (oracle selection, near_tie)."""
+    s_gpu = np.asarray(s_gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.all(np.abs(s_gpu - ref) <= bound), f"{what}: scores outside the rounding bound"
+    ref_idx = orc.topk(ref, k)
+    if np.array_equal(idx, ref_idx):
+        return ref_idx, False
+    diff = float(np.max(np.abs(s_gpu - ref)))
+    srt = np.sort(ref)[::-1]
+    assert srt.size > k and srt[k - 1] - srt[k] <= 2 * diff, f"{what}: selection differs beyond a near-tie"
+    sel = idx[idx >= 0]
+    mask = np.zeros(ref.size, bool)
+    mask[sel] = True
+    assert ref[sel].min() + 2 * diff >= ref[~mask].max(), f"{what}: selection not a top-k within the difference"
+    return ref_idx, True
 
 
 def bf16_score_bound(qI, w, kI):

@@ -14,8 +14,9 @@ sides get the same values.  Every stage is then checked against the oracle:
   * attention and its LSE within 1e-4 on the oracle's entries and selection;
   * the grouped projection within 1e-4 on the oracle's attention output;
   * the whole chain run on the GPU's own intermediates: the selection equals the
-    oracle's for every query whose k-th score gap exceeds the effect of the compressors'
-    rounding, and the projected output is within 1e-4 for those queries.
+    oracle's except where the oracle's k-th score gap is within the effect of the
+    compressors' rounding (counted), and the projected output is within 1e-4 wherever the
+    selections agree.
 """
 import math
 
@@ -23,7 +24,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close_abs
+from helpers import assert_close_abs, selection_against_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -141,7 +142,10 @@ def test_c1_chain(L, orc):
     idx_c = idx_c[0].cpu().numpy()
     # When the keys move by at most eps, a score moves by at most
     #   sum_h |w_h| (eps sum_d |qI_hd| + (d_I+1) 2^-23 sum_d |qI_hd||k_d|) + (H_I+1) 2^-23 sum_h |w_h||dot_h|
-    # (the key change, and a rounding of each fma chain that may land differently).
+    # (the key change, and a rounding of each fma chain that may land differently).  The
+    # chain's scores must lie within that bound of the oracle's, and its selection must equal
+    # the oracle's unless the oracle's k-th gap is within twice the largest actual difference.
+    sc_c = sc_c[0].cpu().numpy()
     kI_gn = kI_g[0].cpu().numpy().astype(np.float64)
     eps = float(np.max(np.abs(kI_gn - kI_ref)))
     ka = np.abs(kI_ref) + eps
@@ -151,16 +155,15 @@ def test_c1_chain(L, orc):
         if n <= K:
             np.testing.assert_array_equal(idx_c[t], ref["idx"][t])
         else:
-            srt = np.sort(ref["scores"][t].astype(np.float64))[::-1]
             qa = np.abs(p["qI"][t]).astype(np.float64)
             wa = np.abs(p["w"][t]).astype(np.float64)
             sabs = ka[:n] @ qa.T                                              # [n, H_I]
             per_key = (eps * qa.sum(axis=1) + (DI + 1) * 2.0 ** -23 * sabs) @ wa + (HI + 1) * 2.0 ** -23 * (sabs @ wa)
-            bound = float(per_key.max())
-            if srt[K - 1] - srt[K] <= 2 * bound:
+            _, nt = selection_against_oracle(orc, sc_c[t, :n], idx_c[t], ref["scores"][t], per_key, K,
+                                             f"chain query {t}")
+            if nt:
                 near.append(t)
                 continue
-            np.testing.assert_array_equal(idx_c[t], ref["idx"][t], err_msg=f"chain selection of query {t}")
         assert_close_abs(y_c[t], ref["y"][t], 1e-4, f"chain output of query {t}")
     print(f"\nC1 chain: {T} queries, {len(near)} near-ties excluded from the chain comparison: {near}")
-    assert len(near) <= 8
+    assert len(near) <= T // 50

@@ -22,7 +22,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close_rel_rms, assert_exact_topk, bf16_score_bound, oracle_pool, topk_gap_ok
+from helpers import assert_close_rel_rms, assert_exact_topk, bf16_score_bound, oracle_pool, selection_against_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -53,21 +53,7 @@ def _np(t):
 
 
 def _selection_against_oracle(orc, s_gpu, idx, ref, bound, k, what):
-    """The GPU scores lie within `bound` of the oracle's.  When the oracle's k-th score gap
-    exceeds twice the largest bound the GPU selection must equal the oracle's; otherwise (a
-    near-tie) it must still be a top-k of the oracle's scores up to the bound.  Returns
-    (oracle selection, near_tie)."""
-    assert np.all(np.abs(s_gpu - ref) <= bound), f"{what}: scores outside the rounding bound"
-    ref_idx = orc.topk(ref, k)
-    if topk_gap_ok(ref, k, float(bound.max())):
-        np.testing.assert_array_equal(idx, ref_idx, err_msg=what)
-        return ref_idx, False
-    sel = idx[idx >= 0]
-    mask = np.zeros(ref.size, bool)
-    mask[sel] = True
-    if not mask.all():
-        assert ref[sel].min() + 2 * bound.max() >= ref[~mask].max(), f"{what}: selection not a top-k within the bound"
-    return ref_idx, True
+    return selection_against_oracle(orc, s_gpu, idx, ref, bound, k, what)
 
 
 def _check_fp32_and_stored(out32, out16, ref, what):

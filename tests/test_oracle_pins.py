@@ -535,3 +535,23 @@ def test_group_oproj_equals_block_diagonal(orc):
     y = orc.group_oproj(o, Wg, Wo)
     ref = o.reshape(-1) @ block_diag(*Wg) @ Wo
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-10)
+
+
+def test_oracle_reentrant_under_threads(orc):
+    """Tests and the CPU baseline run the oracle on several threads at once: concurrent
+    top-k and score calls return exactly what sequential ones do."""
+    from concurrent.futures import ThreadPoolExecutor
+    rows = [synth.normal(f"pin.mt.{i}", 20000).astype(np.float32) for i in range(24)]
+    ref = [orc.topk(r, 300) for r in rows]
+    with ThreadPoolExecutor(8) as ex:
+        got = list(ex.map(lambda r: orc.topk(r, 300), rows * 3))
+    for i, g in enumerate(got):
+        np.testing.assert_array_equal(g, ref[i % len(rows)])
+    q = synth.normal("pin.mt.q", (4, 32)).astype(np.float32)
+    w = synth.normal("pin.mt.w", 4).astype(np.float32)
+    ks = [synth.normal(f"pin.mt.k{i}", (500, 32)).astype(np.float32) for i in range(8)]
+    ref_s = [orc.index_scores_f32(q, w, k) for k in ks]
+    with ThreadPoolExecutor(8) as ex:
+        got_s = list(ex.map(lambda k: orc.index_scores_f32(q, w, k), ks * 3))
+    for i, g in enumerate(got_s):
+        np.testing.assert_array_equal(g, ref_s[i % len(ks)])
