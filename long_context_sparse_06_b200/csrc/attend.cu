@@ -55,6 +55,8 @@ constexpr int kMaxSplits = 16;                // row-list splits per query (merg
 constexpr int kOPitchF32 = kDv * 4 + 16;      // staged O rows (padded)
 constexpr int kOPitchBF16 = kDv * 2 + 16;
 static_assert(kH * kOPitchF32 <= 2 * kStageBytes, "staged O fits in the stages");
+static_assert(kH * kOPitchF32 + 4 * (2 * kH + kH / 2 * (kMaxSplits + 2)) <= 2 * kStageBytes,
+              "staged O, (m, l) and the merge weights fit in the stages");
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
@@ -187,7 +189,7 @@ template <bool FP8>
 __global__ void __launch_bounds__(kAtThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_c,
                      const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_cr,
-                     const __grid_constant__ CUtensorMap map_wr, const AttendArgs a, int splits,
+                     const __grid_constant__ CUtensorMap map_wr, const AttendArgs a, int splits, int cmerge,
                      float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ AtBars bars;
@@ -195,6 +197,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     uint8_t* q_s = smem;
     uint8_t* stage_s = smem + kQBytes;
     uint8_t* plo_s = stage_s + 2 * kStageBytes;   // low bf16 part of P (one block)
+    // with the in-cluster split merge: this split's (m, l) per head beside its staged O
+    float* ml_s = reinterpret_cast<float*>(stage_s + kH * kOPitchF32);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g = blockIdx.x / splits;
@@ -635,7 +639,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 if (a.lse != nullptr)
                     a.lse[g * kH + head] = (l_sum > 0.f) ? (m_used + log2f(l_sum)) / kLog2e : -INFINITY;
             } else {
-                float* ml = part_ml + ((g * splits + sp) * kH + head) * 2;
+                float* ml = cmerge ? ml_s + 2 * head : part_ml + ((g * splits + sp) * kH + head) * 2;
                 ml[0] = (l_sum > 0.f) ? m_used : -INFINITY;
                 ml[1] = l_sum;
             }
@@ -644,7 +648,58 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    {
+    if (cmerge) {
+        // ---- split merge inside the query's cluster: split sp (= cluster rank) merges the
+        // heads sp, sp + splits, ... from every split's staged fp32 O and (m, l), read over
+        // distributed shared memory, weights exp2(m_s - M) / L summed in split order.
+        cluster_sync_all();   // every split has staged its partial
+        constexpr int kW = kMaxSplits + 2;
+        float* wt = ml_s + 2 * kH;   // [heads of this split][f_0 .. f_{splits-1}, 1/L]
+        const int nh = (kH - sp + splits - 1) / splits;
+        if ((int)threadIdx.x < nh) {
+            const int h = sp + (int)threadIdx.x * splits;
+            float M = -INFINITY;
+            for (int r = 0; r < splits; ++r) {
+                const float m = ld_dsmem_f32(dsmem_addr(ml_s + 2 * h, (uint32_t)r));
+                const float l = ld_dsmem_f32(dsmem_addr(ml_s + 2 * h + 1, (uint32_t)r));
+                if (l > 0.f) M = fmaxf(M, m);
+            }
+            float L = 0.f;
+            for (int r = 0; r < splits; ++r) {
+                const float m = ld_dsmem_f32(dsmem_addr(ml_s + 2 * h, (uint32_t)r));
+                const float l = ld_dsmem_f32(dsmem_addr(ml_s + 2 * h + 1, (uint32_t)r));
+                const float f = l > 0.f ? exp2f(m - M) : 0.f;
+                wt[threadIdx.x * kW + r] = f;
+                L += l * f;
+            }
+            wt[threadIdx.x * kW + kMaxSplits] = L > 0.f ? 1.f / L : 0.f;
+            if (a.lse != nullptr) a.lse[g * kH + h] = L > 0.f ? (M + log2f(L)) / kLog2e : -INFINITY;
+        }
+        __syncthreads();
+        for (int it = (int)threadIdx.x; it < nh * (kDv / 4); it += kAtThreads) {
+            const int i = it / (kDv / 4), q4 = it - i * (kDv / 4);
+            const int h = sp + i * splits;
+            const float* rw = wt + i * kW;
+            const uint8_t* src = stage_s + h * kOPitchF32 + q4 * 16;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int r = 0; r < splits; ++r) {
+                const float4 v = ld_dsmem_f4(dsmem_addr(src, (uint32_t)r));
+                const float f = rw[r];
+                acc.x += v.x * f;
+                acc.y += v.y * f;
+                acc.z += v.z * f;
+                acc.w += v.w * f;
+            }
+            const float iv = rw[kMaxSplits];
+            const int64_t o4 = (g * kH + h) * (kDv / 4) + q4;
+            if (a.out_dtype == LCS_F32)
+                reinterpret_cast<float4*>(a.out)[o4] = make_float4(acc.x * iv, acc.y * iv, acc.z * iv, acc.w * iv);
+            else
+                reinterpret_cast<uint2*>(a.out)[o4] =
+                    make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv), pack_bf16x2(acc.z * iv, acc.w * iv));
+        }
+        cluster_sync_all();   // no CTA leaves while a peer still reads its staged partial
+    } else {
         // the staged O rows (normalised output, or this split's fp32 partial) go out with
         // coalesced 16-byte stores from every thread of the CTA
         const bool f32 = splits > 1 || a.out_dtype == LCS_F32;
@@ -838,6 +893,39 @@ int choose_splits(const AttendArgs& a) {
     return best;
 }
 
+// The in-cluster split merge is used when a query's splits fit one portable cluster and all
+// of the launch's clusters can be resident at once (checked once per kernel and split count).
+bool cluster_merge_ok(const void* kern, int splits, int64_t queries) {
+    if (splits < 2 || splits > 8) return false;
+    static std::mutex mu;
+    static const void* kerns[2] = {nullptr, nullptr};
+    static int cache[2][9];
+    std::lock_guard<std::mutex> lock(mu);
+    int slot = kerns[0] == kern ? 0 : kerns[1] == kern ? 1 : (kerns[0] == nullptr ? 0 : 1);
+    if (kerns[slot] != kern) {
+        kerns[slot] = kern;
+        for (int i = 0; i < 9; ++i) cache[slot][i] = 0;
+    }
+    if (cache[slot][splits] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)splits);
+        cfg.blockDim = dim3(kAtThreads);
+        cfg.dynamicSmemBytes = kAtSmem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)splits;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+        cudaGetLastError();
+        cache[slot][splits] = n > 0 ? n : -1;
+    }
+    return cache[slot][splits] >= queries;
+}
+
 }  // namespace
 
 // Split partials: fp32 O [queries, splits, 64, 512] and (m, l) [queries, splits, 64, 2].
@@ -909,9 +997,30 @@ cudaError_t launch_attend(const AttendArgs& a, void* scratch, int* status, cudaS
         part_o = static_cast<float*>(scratch);
         part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256(queries * splits * kH * kDv * 4));
     }
-    e = launch_k(kern, dim3((unsigned)(queries * splits)), dim3(kAtThreads), kAtSmem, s, pdl, mq, mc, mw, mcr, mwr, a, splits,
-                 part_o, part_ml, status);
-    if (e != cudaSuccess || splits == 1) return e;
+    const int cmerge = cluster_merge_ok(reinterpret_cast<const void*>(kern), splits, queries) ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(queries * splits));
+    cfg.blockDim = dim3(kAtThreads);
+    cfg.dynamicSmemBytes = kAtSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (cmerge) {   // a query's splits form one cluster and merge their partials in shared memory
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)splits;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mc, mw, mcr, mwr, a, splits, cmerge, part_o, part_ml, status);
+    if (e != cudaSuccess || splits == 1 || cmerge) return e;
     return launch_k(attend_combine_kernel, dim3((unsigned)(queries * kH)), dim3(128), 0, s, true, part_o, part_ml,
                     splits, a.out, a.out_dtype, a.lse);
 }

@@ -10,8 +10,8 @@
 // element is ranked by the 64-bit composite (key << 32 | ~index), so "larger
 // composite" is exactly "larger score, then lower index".
 //
-// Rows of at most 32768 entries (decode over 128K tokens, the tiny prefill): one CTA of
-// 1024 threads per row with the whole row in registers and an exact radix select
+// Few rows of at most 65536 entries (decode over 128K tokens, the tiny prefill): a cluster
+// of up to 8 CTAs per row with the whole row in registers and an exact radix select
 // (topk_row_kernel, below).  Longer rows: one CTA of 512 threads per query row, or a
 // cluster of them per row when there are few rows:
 //  1. Lower bound: a fixed strided sample of 512 keys is histogrammed over the
@@ -495,27 +495,40 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
 }
 
 // ------------------------------------------------------ rows held in registers
-// Rows of at most kRowT * kRowKPT entries: one CTA of kRowT threads per row, thread t
-// holding the kRowKPT consecutive keys starting at t * kRowKPT (so thread order is index
-// order), in registers and mirrored in shared memory for the passes that visit only a
-// thread's remaining candidates (a 32-bit mask per thread).  An exact MSB-first radix select finds the k-th largest key:
-// each pass histograms the next digit of the keys that still share the resolved prefix,
-// and a block scan from the top bin finds the digit holding the k-th; the select stops
-// early once the remaining count equals that bin's population (the whole bin is taken).
-// One more block scan then places every selected key: all keys above the threshold, and
-// the lowest-index ones equal to it, in ascending index order.
-constexpr int kRowT = 1024, kRowKPT = 32, kRowBins = 2048;
+// Rows of at most kRowMaxP * kRowT * kRowKPT entries: a cluster of P CTAs per row (P the
+// fewest that hold the row), CTA r of kRowT threads holding entries [r * kRowT * kRowKPT,
+// ...), thread t the kRowKPT consecutive keys from t * kRowKPT of its part -- in registers,
+// and mirrored in shared memory for the passes that visit only a thread's remaining
+// candidates (a bit mask per thread).  Cluster order, then thread order, is index order.
+// An exact MSB-first radix select finds the k-th largest key: each pass histograms the next
+// digit of the keys that still share the resolved prefix, every CTA sums the cluster's
+// histograms over distributed shared memory, and the same block scan in every CTA picks the
+// digit holding the k-th; the select stops early once the remaining count equals that
+// bin's population (the whole bin is taken).  A last exchange of per-CTA counts places every
+// selected key: all keys above the threshold, and the lowest-index ones equal to it, in
+// ascending index order.
+constexpr int kRowT = 512, kRowKPT = 16, kRowBins = 2048, kRowMaxP = 8;
+constexpr int kRowPart = kRowT * kRowKPT;   // 8192 entries per CTA
+
+struct RowSmem {
+    uint32_t ks[kRowKPT * kRowT];           // key j of thread t at ks[j * kRowT + t]
+    uint32_t hist[kRowBins];                // this CTA's histogram (read by the peers)
+    uint32_t ghist[kRowBins];               // the cluster's histogram
+    uint32_t wsum[2][32];
+    uint32_t cnt[2];                        // this CTA's keys above / tied (read by the peers)
+    uint32_t s_digit, s_above, s_inbin;
+};
 
 template <bool BF16>
 __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restrict__ scores, int64_t N_c,
                                                             const int64_t* __restrict__ q_pos, int m, int k,
-                                                            int32_t* __restrict__ idx_out) {
-    extern __shared__ uint32_t ks[];   // [kRowKPT][kRowT]: key j of thread t at ks[j * kRowT + t]
-    __shared__ uint32_t hist[kRowBins];
-    __shared__ uint32_t wsum[2][32];
-    __shared__ uint32_t s_digit, s_above, s_inbin;
+                                                            int32_t* __restrict__ idx_out, int P) {
+    extern __shared__ __align__(16) uint8_t row_smem_raw[];
+    RowSmem& sm = *reinterpret_cast<RowSmem*>(row_smem_raw);
     constexpr int kBits = BF16 ? 16 : 32;
-    const int64_t row = blockIdx.x;
+    constexpr int kWarpsR = kRowT / 32;
+    const int64_t row = blockIdx.x / P;
+    const int rank = (int)(blockIdx.x - row * P);   // == rank in the row's cluster
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     int64_t n = N_c;
     if (q_pos != nullptr) {
@@ -530,13 +543,14 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #endif
 
-    if (n <= k) {
-        for (int i = t; i < k; i += kRowT) out[i] = (i < n) ? i : -1;
+    if (n <= k) {   // the same decision in every CTA of the cluster
+        if (rank == 0)
+            for (int i = t; i < k; i += kRowT) out[i] = (i < n) ? i : -1;
         return;
     }
 
     // ---- keys of this thread (entries at or beyond n read as key 0, below every finite score)
-    const int64_t base = (int64_t)t * kRowKPT;
+    const int64_t base = (int64_t)rank * kRowPart + (int64_t)t * kRowKPT;
     uint32_t key[kRowKPT];
     const bool vec = (reinterpret_cast<uintptr_t>(srow) & 15) == 0 && base + kRowKPT <= n;
     if (vec) {
@@ -562,15 +576,11 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
 #pragma unroll
         for (int j = 0; j < kRowKPT; ++j) key[j] = (base + j < n) ? load_key<BF16>(srow, base + j) : 0u;
     }
-#pragma unroll
-    for (int j = 0; j < kRowKPT; ++j) ks[j * kRowT + t] = key[j];
 
-    // ---- radix select: digits of 11, 11, 10 bits (fp32 keys) or 11, 5 (bf16 keys).  After
-    // each pass the thread keeps a mask of its keys that still share the resolved prefix, so
-    // later passes and the placement visit only those.
+    // ---- radix select: digits of 11, 11, 10 bits (fp32 keys) or 11, 5 (bf16 keys)
     uint32_t prefix = 0, krem = (uint32_t)k;
-    uint32_t cand = 0xFFFFFFFFu;   // keys still sharing the prefix (all of them before pass 0)
-    uint32_t above = 0;            // keys already known to lie above the threshold
+    uint32_t cand = (1u << kRowKPT) - 1u;   // keys still sharing the prefix
+    uint32_t above = 0;                     // keys known to lie above the threshold
     int done = 0;
     bool whole_bin = false;
 #pragma unroll 1
@@ -578,61 +588,79 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
         const int width = (kBits - done) < 11 ? (kBits - done) : 11;
         const int shift = kBits - done - width;
         const int nb = 1 << width;
-        for (int i = t; i < nb; i += kRowT) hist[i] = 0;
+        for (int i = t; i < nb; i += kRowT) sm.hist[i] = 0;
         __syncthreads();
         if (pass == 0) {
 #pragma unroll
-            for (int j = 0; j < kRowKPT; ++j) atomicAdd(&hist[key[j] >> shift], 1u);
+            for (int j = 0; j < kRowKPT; ++j) atomicAdd(&sm.hist[key[j] >> shift], 1u);
         } else {
-            for (uint32_t m = cand; m != 0; m &= m - 1) {
-                const uint32_t kk = ks[(__ffs(m) - 1) * kRowT + t];
-                atomicAdd(&hist[(kk >> shift) & (nb - 1)], 1u);
+            for (uint32_t mm = cand; mm != 0; mm &= mm - 1) {
+                const uint32_t kk = sm.ks[(__ffs(mm) - 1) * kRowT + t];
+                atomicAdd(&sm.hist[(kk >> shift) & (nb - 1)], 1u);
             }
         }
+        // the cluster's histogram: every CTA sums all P parts in rank order
+        if (P > 1) cluster_sync_all();
+        else __syncthreads();
+        for (int i = t; i < nb; i += kRowT) {
+            uint32_t v = 0;
+            for (int r = 0; r < P; ++r)
+                v += (r == rank) ? sm.hist[i] : ld_dsmem_u32(dsmem_addr(&sm.hist[i], (uint32_t)r));
+            sm.ghist[i] = v;
+        }
         __syncthreads();
-        // bins from the top: thread t owns bins nb-1-2t and nb-2-2t (nb = 2048), or nb-1-t
-        const int per = nb >= 2 * kRowT ? 2 : 1;
+        // bins from the top: thread t owns bins b0, b0-1, ... (per of them; per = nb / kRowT
+        // for nb = 2048, else 1)
+        const int per = nb > kRowT ? nb / kRowT : 1;
         const int b0 = nb - 1 - t * per;
-        uint32_t c0 = 0, c1 = 0;
-        if (b0 >= 0) c0 = hist[b0];
-        if (per == 2 && b0 >= 1) c1 = hist[b0 - 1];
-        const uint32_t local = c0 + c1;
+        uint32_t c[4] = {0u, 0u, 0u, 0u};
+        uint32_t local = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (u < per && b0 - u >= 0) {
+                c[u] = sm.ghist[b0 - u];
+                local += c[u];
+            }
         uint32_t incl = local;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        if (lane == 31) wsum[0][warp] = incl;
+        if (lane == 31) sm.wsum[0][warp] = incl;
         __syncthreads();
         if (warp == 0) {
-            const uint32_t v = wsum[0][lane];
+            const uint32_t v = lane < kWarpsR ? sm.wsum[0][lane] : 0u;
             uint32_t x = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
                 if (lane >= o) x += y;
             }
-            wsum[1][lane] = x - v;
+            sm.wsum[1][lane] = x - v;
         }
         __syncthreads();
-        const uint32_t excl = wsum[1][warp] + incl - local;
-        if (excl < krem && excl + local >= krem) {
-            if (excl + c0 >= krem) {
-                s_digit = (uint32_t)b0;
-                s_above = excl;
-                s_inbin = c0;
-            } else {
-                s_digit = (uint32_t)(b0 - 1);
-                s_above = excl + c0;
-                s_inbin = c1;
-            }
+        uint32_t run = sm.wsum[1][warp] + incl - local;
+        if (run < krem && run + local >= krem) {
+            bool found = false;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (!found && u < per) {
+                    if (run + c[u] >= krem) {
+                        sm.s_digit = (uint32_t)(b0 - u);
+                        sm.s_above = run;
+                        sm.s_inbin = c[u];
+                        found = true;
+                    } else {
+                        run += c[u];
+                    }
+                }
         }
         __syncthreads();
-        const uint32_t dg = s_digit;
+        const uint32_t dg = sm.s_digit;
         prefix = (prefix << width) | dg;
         done += width;
-        krem -= s_above;
+        krem -= sm.s_above;
         // split this thread's candidates: digit above the threshold digit, or equal to it
         uint32_t nc = 0;
         if (pass == 0) {
@@ -641,17 +669,22 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
                 const uint32_t d = key[j] >> shift;
                 above |= (d > dg ? 1u : 0u) << j;
                 nc |= (d == dg ? 1u : 0u) << j;
+                if (d == dg) sm.ks[j * kRowT + t] = key[j];   // mirrored only where later passes look
             }
         } else {
-            for (uint32_t m = cand; m != 0; m &= m - 1) {
-                const int j = __ffs(m) - 1;
-                const uint32_t d = (ks[j * kRowT + t] >> shift) & (nb - 1);
+            for (uint32_t mm = cand; mm != 0; mm &= mm - 1) {
+                const int j = __ffs(mm) - 1;
+                const uint32_t d = (sm.ks[j * kRowT + t] >> shift) & (nb - 1);
                 if (d > dg) above |= 1u << j;
                 else if (d == dg) nc |= 1u << j;
             }
         }
         cand = nc;
-        if (s_inbin == krem) {   // the whole threshold bin is taken
+        const bool whole = sm.s_inbin == krem;
+        // the peers have read this CTA's histogram before it is cleared again
+        if (P > 1) cluster_sync_all();
+        else __syncthreads();
+        if (whole) {   // the whole threshold bin is taken
             whole_bin = true;
             break;
         }
@@ -669,14 +702,14 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
             ie += ye;
         }
     }
-    __syncthreads();   // wsum is reused
     if (lane == 31) {
-        wsum[0][warp] = ig;
-        wsum[1][warp] = ie;
+        sm.wsum[0][warp] = ig;
+        sm.wsum[1][warp] = ie;
     }
     __syncthreads();
     if (warp == 0) {
-        const uint32_t vg = wsum[0][lane], ve = wsum[1][lane];
+        const uint32_t vg = lane < kWarpsR ? sm.wsum[0][lane] : 0u;
+        const uint32_t ve = lane < kWarpsR ? sm.wsum[1][lane] : 0u;
         uint32_t xg = vg, xe = ve;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -688,22 +721,36 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
             }
         }
         __syncwarp();
-        wsum[0][lane] = xg - vg;
-        wsum[1][lane] = xe - ve;
+        if (lane < kWarpsR) {
+            sm.wsum[0][lane] = xg - vg;
+            sm.wsum[1][lane] = xe - ve;
+        }
+        if (lane == 31) {   // this CTA's totals, for the peers of higher rank
+            sm.cnt[0] = xg;
+            sm.cnt[1] = xe;
+        }
     }
-    __syncthreads();
-    const uint32_t gt_before = wsum[0][warp] + ig - gt;
-    const uint32_t e0 = wsum[1][warp] + ie - eq;          // ties before this thread's keys
+    if (P > 1) cluster_sync_all();
+    else __syncthreads();
+    uint32_t cg = 0, ce = 0;   // keys above / tied in the CTAs of lower rank
+    for (int r = 0; r < rank; ++r) {
+        cg += ld_dsmem_u32(dsmem_addr(&sm.cnt[0], (uint32_t)r));
+        ce += ld_dsmem_u32(dsmem_addr(&sm.cnt[1], (uint32_t)r));
+    }
+    const uint32_t gt_before = cg + sm.wsum[0][warp] + ig - gt;
+    const uint32_t e0 = ce + sm.wsum[1][warp] + ie - eq;   // ties before this thread's keys
     uint32_t take = above;
     if (whole_bin) {
         take |= cand;
     } else if (e0 < krem) {   // the first krem - e0 ties of this thread
-        uint32_t m = cand;
-        for (uint32_t r = e0; r < krem && m != 0; ++r) m &= m - 1;
-        take |= cand & ~m;
+        uint32_t mm = cand;
+        for (uint32_t r = e0; r < krem && mm != 0; ++r) mm &= mm - 1;
+        take |= cand & ~mm;
     }
     uint32_t pos = gt_before + (whole_bin ? e0 : (e0 < krem ? e0 : krem));
-    for (uint32_t m = take; m != 0; m &= m - 1) out[pos++] = (int32_t)(base + __ffs(m) - 1);
+    for (uint32_t mm = take; mm != 0; mm &= mm - 1) out[pos++] = (int32_t)(base + __ffs(mm) - 1);
+    // no CTA leaves while a peer may still read its counts
+    if (P > 1) cluster_sync_all();
 }
 
 }  // namespace
@@ -755,12 +802,34 @@ int choose_ranks(int64_t rows, int64_t N_c) {
 template <bool BF16>
 cudaError_t launch_topk_t(const void* scores, int64_t rows, int64_t N_c, const int64_t* q_pos, int m, int k,
                           int32_t* idx, cudaStream_t s, bool pdl) {
-    if (N_c <= (int64_t)kRowT * kRowKPT) {   // the whole row fits one CTA's registers
-        constexpr size_t smem = sizeof(uint32_t) * kRowT * kRowKPT;
+    // The whole row fits a cluster's registers, and the clusters fit about two waves: few long
+    // rows (decode).  Many rows (prefill) go to the kernel below, one CTA per row.
+    const int P_row = (int)((N_c + kRowPart - 1) / kRowPart);
+    if (N_c <= (int64_t)kRowMaxP * kRowPart && rows * P_row <= 2 * (int64_t)num_sms()) {
+        const int P = P_row;
+        constexpr size_t smem = sizeof(RowSmem);
         cudaError_t e = set_smem_once(reinterpret_cast<const void*>(topk_row_kernel<BF16>), smem);
         if (e != cudaSuccess) return e;
-        return launch_k(topk_row_kernel<BF16>, dim3((unsigned)rows), dim3(kRowT), smem, s, pdl, scores, N_c, q_pos, m,
-                        k, idx);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(rows * P));
+        cfg.blockDim = dim3(kRowT);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[2];
+        int na = 0;
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)P;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+        if (pdl) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        return cudaLaunchKernelEx(&cfg, topk_row_kernel<BF16>, scores, N_c, q_pos, m, k, idx, P);
     }
     const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16>);
     cudaError_t e = set_smem_once(kern, sizeof(TopkSmem));

@@ -128,7 +128,7 @@ def test_topk_bit_exact_on_same_scores(L, orc, dtype, N):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("N", [32768, 32769])   # the longest row held in registers, and one more
+@pytest.mark.parametrize("N", [8192, 32768, 40000, 65536, 65537])   # 1, 4, 5 and 8 CTAs per row; one more
 def test_topk_register_rows(L, orc, dtype, N):
     """Rows at the register-resident limit: ties at the threshold, all-equal rows, monotone
     rows, +-0, a threshold bin crowded to its last bits, and causal availability."""
