@@ -17,7 +17,9 @@
 //      S [64 heads x 64 rows] = Q [64 x 576] . K_chunk^T        (K-major x K-major)
 //    warp 13 issues
 //      O [64 heads x 512]    += P [64 x 64 rows] . V_chunk       (K-major x MN-major)
-//    with P = P_hi + P_lo, two bf16 parts, so P.V is two MMAs per chunk.  O lives in
+//    with P in bf16: for FP8 rows P = P_hi + P_lo, two bf16 parts (two MMAs per K step);
+//    for bf16 rows a single part, and the softmax of chunk c+1 then runs under the P.V of
+//    chunk c (it waits for that P.V only to rescale O).  O lives in
 //    TMEM as two interleaved M=64 accumulators (dims 0-255 in lanes 0-15 of each
 //    32-lane quarter, dims 256-511 in lanes 16-31), S double-buffered beside it;
 //  * warps 4-11 fill a 2-stage ring, four warps per stage, writing the SW128 layout that
@@ -29,8 +31,8 @@
 //    window chunks are fetched before the kernel waits for the preceding kernel
 //    (programmatic dependent launch): they do not depend on it;
 //  * warps 0-3 run the online softmax on S (fp32, exp2), write P_hi into the chunk's
-//    RoPE column block (dead once Q.K^T has read it) and P_lo into a block of its
-//    own, rescale O in TMEM only when a head's running max grows by more than 2^8
+//    RoPE column block (dead once Q.K^T has read it) and, for FP8 rows, P_lo into a block of
+//    its own, rescale O in TMEM only when a head's running max grows by more than 2^8
 //    in weight, and write O / l out through shared memory (coalesced);
 //  * with several splits each CTA writes its unnormalised O and (m, l) to the
 //    workspace, and attend_combine_kernel merges them in split order.
@@ -474,7 +476,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                         const uint32_t od = tmem + (half ? (16u << 16) : 0u);
                         const uint64_t vk = vd + (uint64_t)((half * 4 * kBlk + kk * 2048) >> 4);
                         mma_bf16_ss(od, pd + (uint64_t)((kk * 32) >> 4), vk, idesc_pv, (c | kk) ? 1u : 0u);
-                        mma_bf16_ss(od, pld + (uint64_t)((kk * 32) >> 4), vk, idesc_pv, 1u);
+                        if constexpr (FP8) mma_bf16_ss(od, pld + (uint64_t)((kk * 32) >> 4), vk, idesc_pv, 1u);
                     }
                 mma_commit(&bars.kempty[st]);
                 mma_commit(&bars.ofull[st]);
@@ -529,11 +531,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 rescale = (c > 0);
                 m_used = m_new;
             }
-            // p = exp2(scale*log2e*s - m) as two bf16 parts, p ~ hi + lo (relative error
-            // about 2^-17; a single bf16 P costs 2^-9 per weight, which heavy-tailed V turns
-            // into output errors near 2e-2 of the output RMS).  hi goes into the chunk's RoPE
-            // column block (dead once Q.K^T has read it), lo into the one P_lo block; both are
-            // K-major SW128 rows of 128 B per head.
+            // p = exp2(scale*log2e*s - m) in bf16 for P.V.  FP8 rows: two bf16 parts, p ~ hi +
+            // lo (relative error about 2^-17; a single bf16 P costs 2^-9 per weight, which the
+            // heavy-tailed values of that format turn into output errors near 2e-2 of the output
+            // RMS).  bf16 rows: the single part hi, and l sums the same rounded weights.  hi goes
+            // into the chunk's RoPE column block (dead once Q.K^T has read it), lo into the one
+            // P_lo block; both are K-major SW128 rows of 128 B per head.
             uint8_t* pblk = stage_s + st * kStageBytes + 8 * kBlk;
             float psum = 0.f;
 #pragma unroll
@@ -547,32 +550,41 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                     pk[q] = pack_bf16x2(p0, p1);
                     const float h0 = bf16_bits_to_f32((uint16_t)(pk[q] & 0xFFFF));
                     const float h1 = bf16_bits_to_f32((uint16_t)(pk[q] >> 16));
-                    sv[j] = __float_as_uint(p0 - h0);          // exact residuals
-                    sv[j + 1] = __float_as_uint(p1 - h1);
-                    psum += p0 + p1;
+                    if constexpr (FP8) {
+                        sv[j] = __float_as_uint(p0 - h0);      // exact residuals
+                        sv[j + 1] = __float_as_uint(p1 - h1);
+                        psum += p0 + p1;
+                    } else {
+                        psum += h0 + h1;
+                    }
                 }
                 *reinterpret_cast<uint4*>(pblk + sw128_off(head, (cbase >> 3) + ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            // P_lo is single-buffered: the previous chunk's P.V must have read it.  (P.V of
+            // The previous chunk's P.V must be complete before P_lo (single-buffered) or O is
+            // written: for FP8 rows every chunk, for bf16 rows only when O is rescaled.  (P.V of
             // chunk c-3 is complete here -- chunk c-1 was gathered after it -- so the
             // per-chunk-parity barrier cannot be two phases behind.)
-            if (c > 0) {
+            const bool any_rescale = __any_sync(0xffffffffu, rescale);
+            if (c > 0 && (FP8 || any_rescale)) {
                 if (!mbar_wait(&bars.ofull[(c - 1) & 1], (uint32_t)(((c - 1) >> 1) & 1), status, 321)) break;
                 tc_fence_after();
             }
+            if constexpr (FP8) {
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t pk[4];
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t pk[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int j = ch * 8 + 2 * q;
-                    pk[q] = pack_bf16x2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                    for (int q = 0; q < 4; ++q) {
+                        const int j = ch * 8 + 2 * q;
+                        pk[q] = pack_bf16x2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                    }
+                    *reinterpret_cast<uint4*>(plo_s + sw128_off(head, (cbase >> 3) + ch)) =
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                *reinterpret_cast<uint4*>(plo_s + sw128_off(head, (cbase >> 3) + ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             psum += __shfl_xor_sync(0xffffffffu, psum, 16);
             l_sum = l_sum * alpha + psum;
-            if (__any_sync(0xffffffffu, rescale)) {
+            if (any_rescale) {
                 // O is stable (the previous chunk's P.V is complete, waited for above).
                 const float f = rescale ? alpha : 1.f;
                 for (int j = 0; j < 256 / 16; ++j) {
