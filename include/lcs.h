@@ -74,6 +74,7 @@ extern "C" {
 #define LCS_OP_ATTEND     2
 #define LCS_OP_DECODE     3
 #define LCS_OP_TOPK       4
+#define LCS_OP_CP_SELECT  5
 
 /*
  * Token compressor, CSA ("DeepSeek V4 深度解析" §2, CSA step 1; "V3 vs V4" page,
@@ -288,6 +289,39 @@ LCS_API int lcs_cache_append(int64_t B, const int64_t* pos, const void* x, const
                  int kv_dtype, int kI_dtype, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Context parallelism for long requests: the compressed entries (and index keys) of every
+ * request are split over G ranks, rank r holding the S entries [offset, offset + S).  One
+ * decode step is, on every rank: csa_index_topk over the rank's entries (local top-k, local
+ * indices), lcs_cp_candidates, an all-gather of the candidates in rank order, lcs_cp_select,
+ * csa_attend over the rank's share of the selection (with lse; the window rows on the rank
+ * that holds them, Tw = 0 elsewhere), an all-gather of (o, lse) in rank order, and
+ * lcs_attn_merge.  The result equals the unsplit step ("DeepSeek V4 深度解析" §2, CSA steps
+ * 2-3): every global top-k entry is in the top-k of its own shard, and candidates gathered in
+ * rank order are in global-index order, so the selection and its tie rule are unchanged; one
+ * softmax over disjoint row sets is the log-sum-exp merge of the parts.
+ *
+ * lcs_cp_candidates: scores [B, S] (LCS_F32 or LCS_BF16; csa_index_topk's scores output),
+ *   idx_local [B, k] (its selection) -> cand_score [B, k] fp32 and cand_idx [B, k] int32
+ *   global index offset + local; -1 entries become (-inf, -1).
+ * lcs_cp_select: cand_score, cand_idx [G, B, k] (all ranks' candidates, rank r at r) ->
+ *   idx_global [B, k] the global top-k (ascending, -1 padded, ties -> lower index) and
+ *   idx_local [B, k] the entries of [offset, offset + S) among them, as local indices
+ *   (ascending, -1 padded: csa_attend's selection form).  Workspace: lcs_workspace_size(
+ *   LCS_OP_CP_SELECT, B, G, 0, 0, k, ...).
+ * lcs_attn_merge: o [G, rows, d_v] fp32 and lse [G, rows] fp32 (rank r's normalised
+ *   attention output and natural-log sum of exp; -inf for an empty row set) -> out
+ *   [rows, d_v] (LCS_F32 or LCS_BF16) = sum_r exp(lse_r - L) o_r with L = log sum_r
+ *   exp(lse_r), summed in rank order; lse_out [rows] = L (or NULL).
+ */
+LCS_API int lcs_cp_candidates(const void* scores, int score_dtype, int64_t B, int64_t S, const int32_t* idx_local,
+                 int k, int64_t offset, float* cand_score, int32_t* cand_idx, cudaStream_t stream);
+LCS_API int lcs_cp_select(const float* cand_score, const int32_t* cand_idx, int G, int64_t B, int k,
+                 int64_t offset, int64_t S, int32_t* idx_global, int32_t* idx_local,
+                 void* ws, size_t ws_bytes, cudaStream_t stream);
+LCS_API int lcs_attn_merge(const float* o, const float* lse, int G, int64_t rows, int d_v, void* out,
+                 int out_dtype, float* lse_out, cudaStream_t stream);
+
+/*
  * Grouped output projection ("DeepSeek V4 深度解析" §2, HCA paragraph: both use a
  * grouped output projection to cut compute; "V3 vs V4" page: 输出端分组投影).
  * The H heads of each token are split into G groups of H/G consecutive heads;
@@ -325,6 +359,7 @@ LCS_API int lcs_quant_fp4(const float* x, int64_t n, int d, void* out, cudaStrea
  * Workspace bytes for op (LCS_OP_*) at the given sizes (unused sizes ignored):
  *   LCS_OP_INDEX_TOPK: B, Q, N_c, k, score_dtype     LCS_OP_TOPK: B, Q, N_c, k
  *   LCS_OP_ATTEND: B, Q, H, d_v (+ N_c, Tw, k for the split plan)
+ *   LCS_OP_CP_SELECT: B, Q = G (ranks), k
  *   LCS_OP_DECODE: everything (both stages)
  * Returns a negative value for invalid sizes.  The first 256 bytes hold the
  * status word; the workspace must be 256-byte aligned.

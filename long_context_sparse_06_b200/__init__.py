@@ -15,13 +15,13 @@ import os
 __all__ = [
     "F32", "BF16", "KV_FP8", "FP4", "MODE_CSA", "MODE_HCA", "LcsError", "lib",
     "csa_compress", "hca_compress", "csa_index_topk", "lcs_topk", "csa_attend", "hca_attend",
-    "decode_fused", "lcs_cache_append", "group_oproj", "lcs_rope", "lcs_quant_kv_fp8", "lcs_quant_fp4",
+    "decode_fused", "lcs_cache_append", "lcs_cp_candidates", "lcs_cp_select", "lcs_attn_merge", "group_oproj", "lcs_rope", "lcs_quant_kv_fp8", "lcs_quant_fp4",
     "lcs_workspace_size", "lcs_status", "lcs_clear_status", "lcs_selftest_wait", "workspace", "kv_fp8_row_bytes",
 ]
 
 F32, BF16, KV_FP8, FP4 = 0, 1, 2, 3
 MODE_CSA, MODE_HCA = 0, 1
-OP_INDEX_TOPK, OP_ATTEND, OP_DECODE, OP_TOPK = 1, 2, 3, 4
+OP_INDEX_TOPK, OP_ATTEND, OP_DECODE, OP_TOPK, OP_CP_SELECT = 1, 2, 3, 4, 5
 # return codes (include/lcs.h)
 LCS_OK, LCS_ERR_INVALID, LCS_ERR_UNSUPPORTED, LCS_ERR_CUDA = 0, -1, -2, -3
 LCS_ERR_TIMEOUT, LCS_ERR_DEVICE, LCS_ERR_WORKSPACE, LCS_ERR_TOO_LARGE = -4, -5, -6, -7
@@ -56,6 +56,9 @@ def lib():
             "hca_attend": [P, I, P, P, I, I64, I64, I64, I64, P, P, I, I, I, I, I, F, P, I, P, P, SZ, P],
             "lcs_cache_append": [I64, P, P, P, I, P, P, P, P, P, P, I, I, I, F, P, P, P, I, P, P, P, I64, I64, I, I,
                                  P, SZ, P],
+            "lcs_cp_candidates": [P, I, I64, I64, P, I, I64, P, P, P],
+            "lcs_cp_select": [P, P, I, I64, I, I64, I64, P, P, P, SZ, P],
+            "lcs_attn_merge": [P, P, I, I64, I, P, I, P, P],
             "decode_fused": [I, I64, P, I, P, P, I, I64, I64, I, I, I, F, P, I, P, P, I, I, I, I, I, P, I, P, P, P,
                              SZ, P],
             "group_oproj": [P, I64, I, I, P, I, I, P, I, P, P],
@@ -323,6 +326,44 @@ def lcs_cache_append(pos, x, kx, z, zI, zh, bias, biasI, biash, raw, logits, win
           _ptr(comp), _ptr(kI), _ptr(hca), N_c, hca.shape[1], kv_dtype, kI_dtype, _ptr(ws), ws.numel(),
           _stream(stream))
     return ws
+
+
+# ------------------------------------------------- context parallelism (one long request)
+def lcs_cp_candidates(scores, idx_local, offset, stream=None):
+    """scores [B, S] (fp32/bf16), idx_local [B, k] -> (cand_score [B, k] fp32, cand_idx [B, k] int32)."""
+    torch = _torch()
+    B, S = scores.shape
+    k = idx_local.shape[-1]
+    cs = torch.empty((B, k), dtype=torch.float32, device=scores.device)
+    ci = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    _call("lcs_cp_candidates", _ptr(scores), _dt(scores), B, S, _ptr(idx_local), k, offset, _ptr(cs), _ptr(ci),
+          _stream(stream))
+    return cs, ci
+
+
+def lcs_cp_select(cand_score, cand_idx, offset, S, ws=None, stream=None):
+    """cand_score, cand_idx [G, B, k] -> (idx_global [B, k], idx_local [B, k])."""
+    torch = _torch()
+    G, B, k = cand_score.shape
+    ig = torch.empty((B, k), dtype=torch.int32, device=cand_score.device)
+    il = torch.empty((B, k), dtype=torch.int32, device=cand_score.device)
+    if ws is None:
+        ws = workspace(lcs_workspace_size(OP_CP_SELECT, B, G, 0, 0, k), cand_score.device)
+    _call("lcs_cp_select", _ptr(cand_score), _ptr(cand_idx), G, B, k, offset, S, _ptr(ig), _ptr(il), _ptr(ws),
+          ws.numel(), _stream(stream))
+    return ig, il
+
+
+def lcs_attn_merge(o, lse, out_dtype=None, want_lse=False, stream=None):
+    """o [G, ..., d_v] fp32, lse [G, ...] fp32 -> out [..., d_v] (and the merged lse)."""
+    torch = _torch()
+    G = o.shape[0]
+    d_v = o.shape[-1]
+    rows = lse[0].numel()
+    out = torch.empty(o.shape[1:], dtype=out_dtype or torch.float32, device=o.device)
+    lo = torch.empty(lse.shape[1:], dtype=torch.float32, device=o.device) if want_lse else None
+    _call("lcs_attn_merge", _ptr(o), _ptr(lse), G, rows, d_v, _ptr(out), _dt(out), _ptr(lo), _stream(stream))
+    return (out, lo) if want_lse else out
 
 
 # --------------------------------------------------------------------- misc

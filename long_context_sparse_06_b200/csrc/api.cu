@@ -502,6 +502,37 @@ int lcs_cache_append(int64_t B, const int64_t* pos, const void* x, const void* k
                                          kI_dtype, status_of(ws), stream));
 }
 
+// ------------------------------------------------- context parallelism (one long request)
+int lcs_cp_candidates(const void* scores, int score_dtype, int64_t B, int64_t S, const int32_t* idx_local, int k,
+                      int64_t offset, float* cand_score, int32_t* cand_idx, cudaStream_t stream) {
+    if (scores == nullptr || idx_local == nullptr || cand_score == nullptr || cand_idx == nullptr) return LCS_ERR_INVALID;
+    if (B < 0 || S < 0 || k < 0 || k > 4096 || offset < 0 || offset + S >= (int64_t(1) << 31)) return LCS_ERR_INVALID;
+    if (score_dtype != LCS_F32 && score_dtype != LCS_BF16) return LCS_ERR_UNSUPPORTED;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    return from_cuda(launch_cp_candidates(scores, score_dtype, B, S, idx_local, k, offset, cand_score, cand_idx, stream));
+}
+
+int lcs_cp_select(const float* cand_score, const int32_t* cand_idx, int G, int64_t B, int k, int64_t offset, int64_t S,
+                  int32_t* idx_global, int32_t* idx_local, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (cand_score == nullptr || cand_idx == nullptr || idx_global == nullptr || idx_local == nullptr)
+        return LCS_ERR_INVALID;
+    if (G < 1 || G > 64 || B < 0 || k < 0 || k > 4096 || offset < 0 || S < 0) return LCS_ERR_INVALID;
+    const int64_t need = kStatusBytes + align256(cp_select_scratch_bytes(G, B, k));
+    if (ws == nullptr || (int64_t)ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)) return LCS_ERR_WORKSPACE;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    return from_cuda(launch_cp_select(cand_score, cand_idx, G, B, k, offset, S, idx_global, idx_local,
+                                      static_cast<uint8_t*>(ws) + kStatusBytes, status_of(ws), stream));
+}
+
+int lcs_attn_merge(const float* o, const float* lse, int G, int64_t rows, int d_v, void* out, int out_dtype,
+                   float* lse_out, cudaStream_t stream) {
+    if (o == nullptr || lse == nullptr || out == nullptr) return LCS_ERR_INVALID;
+    if (G < 1 || G > 1024 || rows < 0 || d_v <= 0 || d_v > 4096) return LCS_ERR_INVALID;
+    if (out_dtype != LCS_F32 && out_dtype != LCS_BF16) return LCS_ERR_UNSUPPORTED;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    return from_cuda(launch_attn_merge(o, lse, G, rows, d_v, out, out_dtype, lse_out, stream));
+}
+
 // ------------------------------------------------------------------- misc
 int group_oproj(const float* o, int64_t T, int H, int d_v, const float* Wg, int G, int d_g, const float* Wo,
                 int hidden, float* y, cudaStream_t stream) {
@@ -540,6 +571,9 @@ int64_t lcs_workspace_size(int op, int64_t B, int64_t Q, int64_t N_c, int64_t Tw
     if (B < 0 || Q < 0 || N_c < 0 || Tw < 0 || k < 0) return -1;
     switch (op) {
         case LCS_OP_TOPK: return kStatusBytes;
+        case LCS_OP_CP_SELECT:   // Q carries the number of ranks G
+            if (Q < 1 || Q > 64) return -1;
+            return kStatusBytes + align256(cp_select_scratch_bytes((int)Q, B, k));
         case LCS_OP_INDEX_TOPK:
             return plan_index(B, Q, N_c, score_dtype, false, score_dtype == LCS_BF16).end;
         case LCS_OP_ATTEND: {

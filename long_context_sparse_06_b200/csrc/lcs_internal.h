@@ -76,6 +76,16 @@ cudaError_t launch_cache_append(const int64_t* pos, const void* x, const void* k
                                 float* logits, void* win, int win_dtype, void* comp, void* kI, void* hca, int64_t B,
                                 int64_t N_c, int64_t N_h, int kv_dtype, int kI_dtype, int* status, cudaStream_t s);
 
+// cp.cu -- context parallelism for one long request (entries split over ranks)
+cudaError_t launch_cp_candidates(const void* scores, int score_dtype, int64_t B, int64_t S, const int32_t* idx_local,
+                                 int k, int64_t offset, float* cand_score, int32_t* cand_idx, cudaStream_t s);
+int64_t cp_select_scratch_bytes(int G, int64_t B, int k);
+cudaError_t launch_cp_select(const float* cand_score, const int32_t* cand_idx, int G, int64_t B, int k, int64_t offset,
+                             int64_t S, int32_t* idx_global, int32_t* idx_local, void* scratch, int* status,
+                             cudaStream_t s);
+cudaError_t launch_attn_merge(const float* o, const float* lse, int G, int64_t rows, int d_v, void* out, int out_dtype,
+                              float* lse_out, cudaStream_t s);
+
 // noalloc.cu -- device address of the fixed scratch array behind csa_attend_noalloc
 // for the current device (looked up once per device).  LCS_OK or LCS_ERR_CUDA.
 int noalloc_scratch(void** ptr);
