@@ -145,6 +145,37 @@ LCS_API int csa_index_topk(const void* qI, int qI_dtype, const float* w, const v
                    int32_t* idx, void* scores, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Compressor with its input projections fused in ("DeepSeek V4 深度解析" §2, CSA step 1:
+ * the pooled KV rows and the per-token pooling logits are linear in the token's hidden
+ * state).  As csa_compress (hca_compress with overlap 0) on
+ *   x[b,t,:] = h[b,t,:] . Wx   and   z[b,t] = h[b,t,:] . wz,
+ * each projected value the fp32 fma chain over the hidden dims in order; the projected rows
+ * stay on chip.
+ *   h [B, T, hidden], h_tail [B, overlap, hidden] or NULL  h_dtype (LCS_F32 or LCS_BF16)
+ *   Wx [hidden, d] h_dtype; wz [hidden] fp32; bias [m + overlap] fp32
+ *   out [B, T/m, d] out_dtype (LCS_F32 or LCS_BF16)
+ * CUDA cores, for small hidden states: LCS_ERR_UNSUPPORTED when one entry's window of hidden
+ * and projected rows, (m + overlap) * (hidden + d + 1) floats, exceeds 150 KB.
+ */
+LCS_API int lcs_compress_proj(const void* h, int h_dtype, int64_t B, int64_t T, int hidden, const void* h_tail,
+                 const void* Wx, int d, const float* wz, const float* bias, int m, int overlap,
+                 int d_rope, float rope_theta, int64_t pos0, void* out, int out_dtype, cudaStream_t stream);
+
+/*
+ * Lightning indexer + top-k with the query projection fused in ("DeepSeek V4 深度解析" §2,
+ * CSA step 2: the index heads and the per-head weights come from the query token's hidden
+ * state).  As csa_index_topk on fp32 keys with
+ *   qI[b,q,:,:] = h[b,q,:] . W_qI   (reshaped [H_I, d_I])   and   w[b,q,:] = h[b,q,:] . W_w,
+ * each the fp32 fma chain over the hidden dims in order, then the fp32 score chains.
+ *   h [B, Q, hidden] fp32; W_qI [hidden, H_I * d_I] fp32; W_w [hidden, H_I] fp32;
+ *   kI [B, N_c, d_I] fp32; q_pos, m, k, idx, scores, ws as csa_index_topk (LCS_F32 scores).
+ * hidden + H_I * (d_I + 1) <= 12288, H_I <= 128, d_I <= 256.
+ */
+LCS_API int csa_index_topk_proj(const float* h, int hidden, const float* W_qI, const float* W_w, const float* kI,
+                 int64_t B, int64_t Q, int64_t N_c, int H_I, int d_I, const int64_t* q_pos, int m, int k,
+                 int32_t* idx, float* scores, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Top-k alone over a given score array (the selection of csa_index_topk).
  *   scores [B, Q, N_c] LCS_F32 or LCS_BF16; q_pos/m as for csa_index_topk;
  *   idx [B, Q, k] int32 (out).

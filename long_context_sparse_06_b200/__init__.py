@@ -14,7 +14,7 @@ import os
 
 __all__ = [
     "F32", "BF16", "KV_FP8", "FP4", "MODE_CSA", "MODE_HCA", "LcsError", "lib",
-    "csa_compress", "hca_compress", "csa_index_topk", "lcs_topk", "csa_attend", "hca_attend",
+    "csa_compress", "hca_compress", "lcs_compress_proj", "csa_index_topk", "csa_index_topk_proj", "lcs_topk", "csa_attend", "hca_attend",
     "decode_fused", "lcs_cache_append", "lcs_cp_candidates", "lcs_cp_select", "lcs_attn_merge", "group_oproj", "lcs_rope", "lcs_quant_kv_fp8", "lcs_quant_fp4",
     "lcs_workspace_size", "lcs_status", "lcs_clear_status", "lcs_selftest_wait", "workspace", "kv_fp8_row_bytes",
 ]
@@ -57,6 +57,8 @@ def lib():
             "lcs_cache_append": [I64, P, P, P, I, P, P, P, P, P, P, I, I, I, F, P, P, P, I, P, P, P, I64, I64, I, I,
                                  P, SZ, P],
             "lcs_cp_candidates": [P, I, I64, I64, P, I, I64, P, P, P],
+            "lcs_compress_proj": [P, I, I64, I64, I, P, P, I, P, P, I, I, I, F, I64, P, I, P],
+            "csa_index_topk_proj": [P, I, P, P, P, I64, I64, I64, I, I, P, I, I, P, P, P, SZ, P],
             "lcs_cp_select": [P, P, I, I64, I, I64, I64, P, P, P, SZ, P],
             "lcs_attn_merge": [P, P, I, I64, I, P, I, P, P],
             "decode_fused": [I, I64, P, I, P, P, I, I64, I64, I, I, I, F, P, I, P, P, I, I, I, I, I, P, I, P, P, P,
@@ -173,7 +175,35 @@ def hca_compress(x, z, bias, m=128, d_rope=0, rope_theta=10000.0, pos0=0, out_dt
     return out
 
 
+def lcs_compress_proj(h, Wx, wz, bias, m=4, overlap=2, d_rope=0, rope_theta=10000.0, pos0=0, h_tail=None,
+                      out_dtype=None, out=None, stream=None):
+    """h [B,T,hidden] (fp32/bf16), Wx [hidden,d] (h's dtype), wz [hidden] fp32 -> [B,T/m,d]."""
+    torch = _torch()
+    B, T, hidden = h.shape
+    d = Wx.shape[1]
+    if out is None:
+        out = torch.empty((B, T // m, d), dtype=out_dtype or h.dtype, device=h.device)
+    _call("lcs_compress_proj", _ptr(h), _dt(h), B, T, hidden, _ptr(h_tail), _ptr(Wx), d, _ptr(wz), _ptr(bias), m,
+          overlap, d_rope, rope_theta, pos0, _ptr(out), _dt(out), _stream(stream))
+    return out
+
+
 # ------------------------------------------------------------------- indexer
+def csa_index_topk_proj(h, W_qI, W_w, kI, k, H_I, q_pos=None, m=4, want_scores=False, ws=None, stream=None):
+    """h [B,Q,hidden] fp32, W_qI [hidden,H_I*d_I], W_w [hidden,H_I], kI [B,N_c,d_I] fp32 ->
+    idx [B,Q,k] (and the scores [B,Q,N_c])."""
+    torch = _torch()
+    B, Q, hidden = h.shape
+    N_c, d_I = kI.shape[1], kI.shape[2]
+    idx = torch.empty((B, Q, k), dtype=torch.int32, device=h.device)
+    scores = torch.empty((B, Q, N_c), dtype=torch.float32, device=h.device) if want_scores else None
+    if ws is None:
+        ws = workspace(lcs_workspace_size(OP_INDEX_TOPK, B, Q, N_c, 0, k), h.device)
+    _call("csa_index_topk_proj", _ptr(h), hidden, _ptr(W_qI), _ptr(W_w), _ptr(kI), B, Q, N_c, H_I, d_I, _ptr(q_pos), m,
+          k, _ptr(idx), _ptr(scores), _ptr(ws), ws.numel(), _stream(stream))
+    return (idx, scores) if want_scores else idx
+
+
 def csa_index_topk(qI, w, kI, k, N_c=None, kI_dtype=None, q_pos=None, m=4, score_dtype=None, want_scores=False,
                    ws=None, stream=None):
     """qI [B,Q,H_I,d_I]; w [B,Q,H_I]; kI [B,N_c,d_I] (fp32/bf16) or FP4 planes (uint8).

@@ -258,6 +258,22 @@ int hca_compress(const void* x, int x_dtype, int64_t B, int64_t T, int d, const 
                            out_dtype, stream);
 }
 
+int lcs_compress_proj(const void* h, int h_dtype, int64_t B, int64_t T, int hidden, const void* h_tail,
+                      const void* Wx, int d, const float* wz, const float* bias, int m, int overlap, int d_rope,
+                      float rope_theta, int64_t pos0, void* out, int out_dtype, cudaStream_t stream) {
+    if (h == nullptr || Wx == nullptr || wz == nullptr || bias == nullptr || out == nullptr) return LCS_ERR_INVALID;
+    if (B < 0 || T < 0 || m < 1 || m > 1024 || overlap < 0 || overlap > 1024 || T % m) return LCS_ERR_INVALID;
+    if (hidden <= 0 || d <= 0 || d > 4096 || d_rope < 0 || d_rope > d || (d_rope & 1)) return LCS_ERR_INVALID;
+    if (overlap == 0 && h_tail != nullptr) return LCS_ERR_INVALID;
+    if (!(rope_theta > 0.f)) return LCS_ERR_INVALID;
+    if ((h_dtype != LCS_F32 && h_dtype != LCS_BF16) || (out_dtype != LCS_F32 && out_dtype != LCS_BF16))
+        return LCS_ERR_UNSUPPORTED;
+    if (compress_proj_tile(hidden, d, m, overlap) == 0) return LCS_ERR_UNSUPPORTED;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    return from_cuda(launch_compress_proj(h, h_dtype, B, T, hidden, h_tail, Wx, d, wz, bias, m, overlap, d_rope,
+                                          rope_theta, pos0, out, out_dtype, stream));
+}
+
 // ------------------------------------------------------------------ indexer
 static int validate_index(const void* qI, int qI_dtype, const float* w, const void* kI, int kI_dtype, int64_t B,
                           int64_t Q, int64_t N_c, int H_I, int d_I, const int64_t* q_pos, int m, int k,
@@ -319,6 +335,25 @@ int csa_index_topk(const void* qI, int qI_dtype, const float* w, const void* kI,
                               g_n_stage_events == 0));
     record_stage(2, stream);
     return r;
+}
+
+int csa_index_topk_proj(const float* h, int hidden, const float* W_qI, const float* W_w, const float* kI, int64_t B,
+                        int64_t Q, int64_t N_c, int H_I, int d_I, const int64_t* q_pos, int m, int k, int32_t* idx,
+                        float* scores, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (h == nullptr || W_qI == nullptr || W_w == nullptr || kI == nullptr || idx == nullptr) return LCS_ERR_INVALID;
+    if (B < 0 || Q < 0 || N_c < 0 || H_I <= 0 || H_I > 128 || d_I <= 0 || d_I > 256 || k < 0 || k > 4096)
+        return LCS_ERR_INVALID;
+    if (hidden <= 0 || hidden > 8192 || (int64_t)hidden + (int64_t)H_I * d_I + H_I > 12288) return LCS_ERR_UNSUPPORTED;
+    if (q_pos == nullptr && Q != 1) return LCS_ERR_INVALID;
+    if (q_pos != nullptr && m < 1) return LCS_ERR_INVALID;
+    if (N_c >= (int64_t(1) << 31) || B * N_c >= (int64_t(1) << 31)) return LCS_ERR_INVALID;
+    const IndexPlan p = plan_index(B, Q, N_c, LCS_F32, scores != nullptr, false);
+    if (ws == nullptr || (int64_t)ws_bytes < p.end || (reinterpret_cast<uintptr_t>(ws) & 255)) return LCS_ERR_WORKSPACE;
+    if (!device_ok()) return LCS_ERR_CUDA;
+    float* sc = scores ? scores : reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p.scores_off);
+    int r = from_cuda(launch_index_proj_f32(h, hidden, W_qI, W_w, kI, B, Q, N_c, H_I, d_I, q_pos, m, sc, stream));
+    if (r != LCS_OK) return r;
+    return from_cuda(launch_topk(sc, LCS_F32, B, Q, N_c, q_pos, m, k, idx, nullptr, status_of(ws), stream, false));
 }
 
 int lcs_topk(const void* scores, int score_dtype, int64_t B, int64_t Q, int64_t N_c, const int64_t* q_pos, int m,

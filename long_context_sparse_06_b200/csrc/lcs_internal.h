@@ -86,6 +86,15 @@ cudaError_t launch_cp_select(const float* cand_score, const int32_t* cand_idx, i
 cudaError_t launch_attn_merge(const float* o, const float* lse, int G, int64_t rows, int d_v, void* out, int out_dtype,
                               float* lse_out, cudaStream_t s);
 
+// proj.cu -- compressor and fp32 indexer with their input projections fused in
+int compress_proj_tile(int hidden, int d, int m, int overlap);
+cudaError_t launch_compress_proj(const void* h, int h_dtype, int64_t B, int64_t T, int hidden, const void* h_tail,
+                                 const void* Wx, int d, const float* wz, const float* bias, int m, int overlap,
+                                 int d_rope, float theta, int64_t pos0, void* out, int out_dtype, cudaStream_t s);
+cudaError_t launch_index_proj_f32(const float* h, int hidden, const float* WqI, const float* Ww, const float* kI,
+                                  int64_t B, int64_t Q, int64_t N_c, int H_I, int d_I, const int64_t* q_pos, int m,
+                                  float* scores, cudaStream_t s);
+
 // noalloc.cu -- device address of the fixed scratch array behind csa_attend_noalloc
 // for the current device (looked up once per device).  LCS_OK or LCS_ERR_CUDA.
 int noalloc_scratch(void** ptr);

@@ -612,6 +612,24 @@ ORC_API void orc_group_oproj(const double* o, const double* Wg, const double* Wo
 /* Array helpers for the Python side (rounding of doubles; code decoding).   */
 /* fmt: 0 fp32, 1 bf16, 2 E4M3 (saturating), 3 E2M1 (saturating).            */
 /* ------------------------------------------------------------------------ */
+/* Projection of a token's hidden state in fp32 ([p3-2] CSA steps 1-2: the  */
+/* KV and index-key rows, the pooling logits, the index queries and head    */
+/* weights are linear in the token's hidden state).  The pages give no      */
+/* order; the order of the fused kernels is adopted: out[t][c] is the fma   */
+/* chain over i = 0 .. n-1 of h[t][i] * W[i][c] in fp32, from 0 (fmaf is    */
+/* correctly rounded).  h [T, n], W [n, d], out [T, d].                      */
+/* ------------------------------------------------------------------------ */
+ORC_API void orc_project_f32(const float* h, const float* W, int64_t T, int n, int d, float* out)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int c = 0; c < d; ++c) {
+            float acc = 0.0f;
+            for (int i = 0; i < n; ++i) acc = fmaf(h[t * n + i], W[(int64_t)i * d + c], acc);
+            out[t * d + c] = acc;
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 ORC_API void orc_round_array(const double* x, int64_t n, int fmt, double* out)
 {
     for (int64_t i = 0; i < n; ++i) {

@@ -74,6 +74,7 @@ def lib():
             "orc_csa_attend": (I64, [P, P, I64, P, I, P, I64, I64, I64, I, I, I, I, D, P, P]),
             "orc_hca_attend": (I64, [P, P, I64, I, P, I64, I64, I64, I, I, I, I, D, P, P]),
             "orc_group_oproj": (None, [P, P, P, I, I, I, I, I, P]),
+            "orc_project_f32": (None, [P, P, I64, I, I, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -386,3 +387,15 @@ def group_oproj(o, Wg, Wo):
     y = np.empty(hidden, np.float64)
     lib().orc_group_oproj(_p(o), _p(Wg), _p(Wo), H, dv, G, dg, hidden, _p(y))
     return y
+
+
+def project_f32(h, W):
+    """fp32 projection of hidden states ("DeepSeek V4 深度解析" §2, CSA steps 1-2: rows, logits,
+    index queries and head weights are linear in the hidden state): out[t, c] is the fp32
+    fma chain over i of h[t, i] * W[i, c], in order.  h [T, n], W [n, d] -> [T, d] float32."""
+    h, W = _f32(h), _f32(W)
+    T, n = h.shape
+    d = W.shape[1]
+    out = np.empty((T, d), np.float32)
+    lib().orc_project_f32(_p(h), _p(W), T, n, d, _p(out))
+    return out

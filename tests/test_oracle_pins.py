@@ -555,3 +555,23 @@ def test_oracle_reentrant_under_threads(orc):
         got_s = list(ex.map(lambda k: orc.index_scores_f32(q, w, k), ks * 3))
     for i, g in enumerate(got_s):
         np.testing.assert_array_equal(g, ref_s[i % len(ks)])
+
+
+def test_project_f32_against_fp64_and_exact_integers(orc):
+    """The fp32 projection: within the fp32 chain's error bound of the fp64 product, exact when
+    every product and partial sum is representable, and each output a chain in input order
+    (a reordered sum would round differently on the cancelling case)."""
+    h = synth.normal("pin.pj.h", (40, 256)).astype(np.float32)
+    W = (synth.normal("pin.pj.w", (256, 36)) / 16).astype(np.float32)
+    got = orc.project_f32(h, W)
+    ref = h.astype(np.float64) @ W.astype(np.float64)
+    bound = 256 * 2.0 ** -24 * (np.abs(h).astype(np.float64) @ np.abs(W).astype(np.float64))
+    assert np.all(np.abs(got - ref) <= bound)
+    hi = np.round(synth.normal("pin.pj.hi", (12, 64)) * 8).astype(np.float32)
+    Wi = np.round(synth.normal("pin.pj.wi", (64, 5)) * 8).astype(np.float32)
+    np.testing.assert_array_equal(orc.project_f32(hi, Wi), (hi.astype(np.float64) @ Wi.astype(np.float64)))
+    # order: 1 + 2^-24 + 2^-24 - 1 in sequence is 0 (each 2^-24 is lost against 1), not 2^-23
+    hc = np.array([[1.0, 2.0 ** -24, 2.0 ** -24, -1.0]], np.float32)
+    Wc = np.ones((4, 1), np.float32)
+    assert orc.project_f32(hc, Wc)[0, 0] == 0.0
+    assert orc.project_f32(hc[:, ::-1].copy(), Wc)[0, 0] == 2.0 ** -23
