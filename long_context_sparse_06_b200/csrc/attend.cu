@@ -27,7 +27,10 @@
 //    P.V): contiguous bf16 chunks (window rows, HCA's compressed rows) with one TMA tile
 //    load per 128-byte column block; selected rows with 16-byte cp.async (row gathers
 //    scale with the number of issuing warps, not with TMA); FP8 rows with
-//    load-convert-store (E4M3 x power-of-two block scale -> bf16, exact).  Q and the
+//    load-convert-store (E4M3 x power-of-two block scale -> bf16, exact).  A stage is
+//    released in two halves (column blocks 0-3 after P.V's first 256 output dims, the
+//    rest after all of it), and a TMA-filled stage lands in the same two halves, so the
+//    next chunk's load and Q.K^T start under the current P.V.  Q and the
 //    window chunks are fetched before the kernel waits for the preceding kernel
 //    (programmatic dependent launch): they do not depend on it;
 //  * warps 0-3 run the online softmax on S (fp32, exp2), write P_hi into the chunk's
@@ -63,9 +66,14 @@ static_assert(kH * kOPitchF32 + 4 * (2 * kH + kH / 2 * (kMaxSplits + 2)) <= 2 * 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;              // log2 of the tolerated growth before O is rescaled
 
+// Each stage is two halves with barriers of their own: column blocks 0-3 (dims 0-255) and
+// blocks 4-8 (dims 256-575; block 8 also carries P after Q.K^T).  P.V releases the first half
+// after its first 256 output dims, and Q.K^T starts on a first half that has landed, so a
+// stage's next load overlaps the rest of its P.V and the next Q.K^T.
+constexpr int kHalfBlocks = 4;   // blocks of the first half
 struct AtBars {
     uint64_t qfull;
-    uint64_t kfull[2], kempty[2];
+    uint64_t kfull[2][2], kempty[2][2];   // [stage][half]
     uint64_t sfull[2], sempty[2];
     uint64_t pfull[2];
     uint64_t ofull[2];   // P.V of chunk c done (per chunk parity)
@@ -211,8 +219,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(&bars.qfull, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars.kfull[i], 128);   // the stage's four producer warps
-            mbar_init(&bars.kempty[i], 1);
+            for (int hf = 0; hf < 2; ++hf) {
+                mbar_init(&bars.kfull[i][hf], 128);   // the stage's four producer warps
+                mbar_init(&bars.kempty[i][hf], 1);
+            }
             mbar_init(&bars.pfull[i], 128);
             mbar_init(&bars.sfull[i], 1);
             mbar_init(&bars.sempty[i], 128);
@@ -287,22 +297,38 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     auto my_row_src = [&](int64_t gc) -> const uint8_t* {
         return (lane < 16 && !contiguous(gc)) ? row_src(gc, pw + 4 * lane) : nullptr;
     };
-    // Fills stage pst with global chunk gc and arrives on kfull (the TMA bytes complete it).
-    auto fill = [&](int64_t gc, const uint8_t* my_src) {
+    // Fills stage pst with global chunk gc (its u-th use; u >= 1 waits for the P.V of the
+    // previous use to release the halves) and arrives on both halves' kfull (the TMA bytes
+    // complete them).  Returns false when a wait ran out.
+    auto wait_half = [&](int u, int hf) -> bool {
+        return u < 1 || group_all(1 + pst, 128, mbar_wait(&bars.kempty[pst][hf], (uint32_t)((u - 1) & 1), status, 310 + hf));
+    };
+    auto fill = [&](int64_t gc, const uint8_t* my_src, int u) -> bool {
         uint8_t* dst = stage_s + pst * kStageBytes;
-        if (contiguous(gc)) {
+        if (contiguous(gc) && !FP8) {
+            // bf16 rows by TMA, half by half: the first half's load starts as soon as P.V has
+            // released it
             const bool w = gc < nwc;
             const int row0 = w ? (int)(b * a.Tw + wp.win_lo + gc * kChunk) : (int)(b * a.N_c + (gc - nwc) * kChunk);
-            if constexpr (!FP8) {
+            for (int hf = 0; hf < 2; ++hf) {
+                if (!wait_half(u, hf)) return false;
+                const int b0 = hf ? kHalfBlocks : 0, b1 = hf ? 9 : kHalfBlocks;
                 if (pw == 0 && lane == 0) {
-                    mbar_arrive_expect_tx(&bars.kfull[pst], kStageBytes);
-                    for (int blk = 0; blk < 9; ++blk)
-                        tma_load_2d(dst + blk * kBlk, w ? &map_w : &map_c, &bars.kfull[pst], blk * 64, row0);
+                    mbar_arrive_expect_tx(&bars.kfull[pst][hf], (b1 - b0) * kBlk);
+                    for (int blk = b0; blk < b1; ++blk)
+                        tma_load_2d(dst + blk * kBlk, w ? &map_w : &map_c, &bars.kfull[pst][hf], blk * 64, row0);
                 } else {
-                    mbar_arrive(&bars.kfull[pst]);
+                    mbar_arrive(&bars.kfull[pst][hf]);
                 }
-                return;
-            } else {
+            }
+            return true;
+        }
+        // every other fill writes the whole stage: wait for both halves first
+        if (!wait_half(u, 0) || !wait_half(u, 1)) return false;
+        if (FP8 && contiguous(gc)) {
+            const bool w = gc < nwc;
+            const int row0 = w ? (int)(b * a.Tw + wp.win_lo + gc * kChunk) : (int)(b * a.N_c + (gc - nwc) * kChunk);
+            {
                 // the codes of column block j (64 rows x 64 B) land in the upper half of
                 // block j, the RoPE dims (bf16, 128-byte swizzle) in block 8; thread tg then
                 // widens 16 codes of rows tg/4 and tg/4 + 32 per block (piece tg%4), reading
@@ -344,8 +370,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                     }
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&bars.kfull[pst]);
-                return;
+                mbar_arrive(&bars.kfull[pst][0]);
+                mbar_arrive(&bars.kfull[pst][1]);
+                return true;
             }
         }
         if constexpr (!FP8) {
@@ -390,7 +417,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&bars.kfull[pst]);
+        mbar_arrive(&bars.kfull[pst][0]);
+        mbar_arrive(&bars.kfull[pst][1]);
+        return true;
     };
     // Window chunks need no selection: the first chunk of each stage is filled before the
     // wait for the preceding kernel when it is a window chunk of this split.
@@ -398,7 +427,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (producer) {
         const int64_t gc = gcof(pst);
         if (gc < nwc) {
-            fill(gc, my_row_src(gc));
+            fill(gc, my_row_src(gc), 0);
             pre = true;
         }
     }
@@ -443,16 +472,22 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             const uint64_t k_desc0 = sw128_desc(smem_u32(stage_s), 16, 1024);
             for (int c = 0; c < nch && ok; ++c) {
                 const int st = c & 1;
-                if (!mbar_wait(&bars.kfull[st], (uint32_t)((c >> 1) & 1), status, 301)) break;
                 if (c >= 2 && !mbar_wait(&bars.sempty[st], (uint32_t)(((c - 2) >> 1) & 1), status, 302)) break;
-                tc_fence_after();
                 const uint64_t kd = k_desc0 + (uint64_t)((st * kStageBytes) >> 4);
+                for (int hf = 0; hf < 2 && ok; ++hf) {   // each half as soon as it has landed
+                    if (!mbar_wait(&bars.kfull[st][hf], (uint32_t)((c >> 1) & 1), status, 301)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int b0 = hf ? kHalfBlocks : 0, b1 = hf ? 9 : kHalfBlocks;
+                    for (int blk = b0; blk < b1; ++blk)
 #pragma unroll
-                for (int blk = 0; blk < 9; ++blk)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(t_s(st), q_desc + (uint64_t)((blk * (kH * 128) + kk * 32) >> 4),
-                                    kd + (uint64_t)((blk * kBlk + kk * 32) >> 4), idesc_qk, (blk | kk) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ss(t_s(st), q_desc + (uint64_t)((blk * (kH * 128) + kk * 32) >> 4),
+                                        kd + (uint64_t)((blk * kBlk + kk * 32) >> 4), idesc_qk, (blk | kk) ? 1u : 0u);
+                }
+                if (!ok) break;
                 mma_commit(&bars.sfull[st]);
             }
         }
@@ -470,7 +505,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 const uint64_t pld = k_desc0 + (uint64_t)((2 * kStageBytes) >> 4);
                 const uint64_t vd = v_desc0 + (uint64_t)((st * kStageBytes) >> 4);
 #pragma unroll
-                for (int half = 0; half < 2; ++half)
+                for (int half = 0; half < 2; ++half) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t od = tmem + (half ? (16u << 16) : 0u);
@@ -478,7 +513,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                         mma_bf16_ss(od, pd + (uint64_t)((kk * 32) >> 4), vk, idesc_pv, (c | kk) ? 1u : 0u);
                         if constexpr (FP8) mma_bf16_ss(od, pld + (uint64_t)((kk * 32) >> 4), vk, idesc_pv, 1u);
                     }
-                mma_commit(&bars.kempty[st]);
+                    // dims 0-255 read blocks 0-3; the second half (blocks 4-7, and P in block 8)
+                    // is released after the rest
+                    mma_commit(&bars.kempty[st][half]);
+                }
                 mma_commit(&bars.ofull[st]);
             }
             mma_commit(&bars.odone);
@@ -491,11 +529,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         for (int c = pst; c < nch; c += 2) {
             const uint8_t* my_src = nxt;
             const int u = c >> 1;
-            // the group leaves together (the FP8 widening syncs on group barriers)
-            if (u >= 1 && !group_all(1 + pst, 128, mbar_wait(&bars.kempty[pst], (uint32_t)((u - 1) & 1), status, 310)))
-                break;
             if (c + 2 < nch) nxt = my_row_src(gcof(c + 2));
-            if (!(pre && c == pst)) fill(gcof(c), my_src);
+            // the group leaves together (its waits are group decisions)
+            if (!(pre && c == pst) && !fill(gcof(c), my_src, u)) break;
         }
     } else if (warp < 4) {
         // ---------------- softmax / correction / epilogue: warps 0..3.  Warp q owns heads
