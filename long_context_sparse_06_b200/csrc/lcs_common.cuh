@@ -232,6 +232,11 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
                  : "memory");
     return v;
 }
+// Remote (or local) shared-memory reduction in a cluster CTA; no value is returned, so the
+// issuing thread does not wait for it.
+__device__ __forceinline__ void red_dsmem_add_u32(uint32_t addr, uint32_t v) {
+    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ unsigned long long ld_dsmem_u64(uint32_t addr) {
     unsigned long long v;
     asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");

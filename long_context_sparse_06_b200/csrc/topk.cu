@@ -502,7 +502,9 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
 // candidates (a bit mask per thread).  Cluster order, then thread order, is index order.
 // An exact MSB-first radix select finds the k-th largest key: each pass histograms the next
 // digit of the keys that still share the resolved prefix, every CTA sums the cluster's
-// histograms over distributed shared memory, and the same block scan in every CTA picks the
+// histograms over distributed shared memory (each CTA adds its nonzero bins into every
+// peer's copy with fire-and-forget remote reductions; the copies are double-buffered, so one
+// cluster barrier per pass suffices), and the same block scan in every CTA picks the
 // digit holding the k-th; the select stops early once the remaining count equals that
 // bin's population (the whole bin is taken).  A last exchange of per-CTA counts places every
 // selected key: all keys above the threshold, and the lowest-index ones equal to it, in
@@ -512,8 +514,8 @@ constexpr int kRowPart = kRowT * kRowKPT;   // 8192 entries per CTA
 
 struct RowSmem {
     uint32_t ks[kRowKPT * kRowT];           // key j of thread t at ks[j * kRowT + t]
-    uint32_t hist[kRowBins];                // this CTA's histogram (read by the peers)
-    uint32_t ghist[kRowBins];               // the cluster's histogram
+    uint32_t hist[kRowBins];                // this CTA's histogram
+    uint32_t ghist[2][kRowBins];            // the cluster's histogram (pass p: buffer p & 1)
     uint32_t wsum[2][32];
     uint32_t cnt[2];                        // this CTA's keys above / tied (read by the peers)
     uint32_t s_digit, s_above, s_inbin;
@@ -577,6 +579,12 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
         for (int j = 0; j < kRowKPT; ++j) key[j] = (base + j < n) ? load_key<BF16>(srow, base + j) : 0u;
     }
 
+    // the first pass's cluster histogram starts cleared in every CTA before any peer adds to it
+    if (P > 1) {
+        for (int i = t; i < kRowBins; i += kRowT) sm.ghist[0][i] = 0;
+        cluster_sync_all();
+    }
+
     // ---- radix select: digits of 11, 11, 10 bits (fp32 keys) or 11, 5 (bf16 keys)
     uint32_t prefix = 0, krem = (uint32_t)k;
     uint32_t cand = (1u << kRowKPT) - 1u;   // keys still sharing the prefix
@@ -588,7 +596,12 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
         const int width = (kBits - done) < 11 ? (kBits - done) : 11;
         const int shift = kBits - done - width;
         const int nb = 1 << width;
+        uint32_t* gh = sm.ghist[pass & 1];
         for (int i = t; i < nb; i += kRowT) sm.hist[i] = 0;
+        // the next pass's buffer: its last readers (this CTA, two passes ago) are done, and
+        // the barrier of this pass orders the clear before any peer's adds to it
+        if (P > 1)
+            for (int i = t; i < kRowBins; i += kRowT) sm.ghist[(pass + 1) & 1][i] = 0;
         __syncthreads();
         if (pass == 0) {
 #pragma unroll
@@ -599,16 +612,19 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
                 atomicAdd(&sm.hist[(kk >> shift) & (nb - 1)], 1u);
             }
         }
-        // the cluster's histogram: every CTA sums all P parts in rank order
-        if (P > 1) cluster_sync_all();
-        else __syncthreads();
-        for (int i = t; i < nb; i += kRowT) {
-            uint32_t v = 0;
-            for (int r = 0; r < P; ++r)
-                v += (r == rank) ? sm.hist[i] : ld_dsmem_u32(dsmem_addr(&sm.hist[i], (uint32_t)r));
-            sm.ghist[i] = v;
-        }
+        // the cluster's histogram: every CTA adds its nonzero bins into every CTA's copy
+        // (integer sums: the order of the additions does not matter)
         __syncthreads();
+        if (P > 1) {
+            for (int i = t; i < nb; i += kRowT) {
+                const uint32_t v = sm.hist[i];
+                if (v != 0)
+                    for (int r = 0; r < P; ++r) red_dsmem_add_u32(dsmem_addr(&gh[i], (uint32_t)r), v);
+            }
+            cluster_sync_all();
+        } else {
+            gh = sm.hist;
+        }
         // bins from the top: thread t owns bins b0, b0-1, ... (per of them; per = nb / kRowT
         // for nb = 2048, else 1)
         const int per = nb > kRowT ? nb / kRowT : 1;
@@ -618,7 +634,7 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             if (u < per && b0 - u >= 0) {
-                c[u] = sm.ghist[b0 - u];
+                c[u] = gh[b0 - u];
                 local += c[u];
             }
         uint32_t incl = local;
@@ -681,9 +697,7 @@ __global__ void __launch_bounds__(kRowT, 1) topk_row_kernel(const void* __restri
         }
         cand = nc;
         const bool whole = sm.s_inbin == krem;
-        // the peers have read this CTA's histogram before it is cleared again
-        if (P > 1) cluster_sync_all();
-        else __syncthreads();
+        __syncthreads();   // s_digit, s_above, s_inbin are rewritten by the next pass
         if (whole) {   // the whole threshold bin is taken
             whole_bin = true;
             break;
