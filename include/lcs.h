@@ -136,8 +136,7 @@ LCS_API int hca_compress(const void* x, int x_dtype, int64_t B, int64_t T, int d
  *                         entries s >= n_avail are unspecified
  * score_dtype: LCS_F32 (kI F32 or BF16) or LCS_BF16 (kI FP4).  d_I % 32 == 0,
  * H_I <= 128 (LCS_F32 path) or H_I == 64 (tensor-core paths).  Tensor-core paths:
- * qI and kI start on a 16-byte boundary, an LCS_FP4 kI on a 32-byte boundary
- * (else LCS_ERR_INVALID).
+ * qI and kI start on a 16-byte boundary (else LCS_ERR_INVALID).
  */
 LCS_API int csa_index_topk(const void* qI, int qI_dtype, const float* w, const void* kI, int kI_dtype,
                    int64_t B, int64_t Q, int64_t N_c, int H_I, int d_I,

@@ -294,8 +294,8 @@ static int validate_index(const void* qI, int qI_dtype, const float* w, const vo
     }
     if (qI_dtype == LCS_BF16 && kI_dtype == LCS_FP4) {
         if (score_dtype != LCS_BF16 || H_I != 64 || d_I != 128) return LCS_ERR_UNSUPPORTED;
-        // the packed key plane is read by TMA in the 16-byte-slot FP4 form, which needs 32 bytes
-        if (!aligned16(qI) || (reinterpret_cast<uintptr_t>(kI) & 31)) return LCS_ERR_INVALID;
+        // the packed key plane is read by TMA as bytes (16-byte aligned base)
+        if (!aligned16(qI) || !aligned16(kI)) return LCS_ERR_INVALID;
         return LCS_OK;
     }
     return LCS_ERR_UNSUPPORTED;

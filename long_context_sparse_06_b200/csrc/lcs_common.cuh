@@ -339,6 +339,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
     return d;
 }
 
+// Shared-memory matrix descriptor, 64-byte swizzle (SW64), sm_100 version 1: K-major rows
+// of 64 bytes in 8-row, 512-byte atoms; sbo = byte stride between 8-row groups (512 for
+// dense atoms), lbo unused.  The start address may step inside an atom (e.g. +32 bytes per
+// K=64 step of packed FP4); the atom base must be 512-byte aligned.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t smem_addr, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFF) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;   // descriptor version (sm_100)
+    d |= (uint64_t)4 << 61;   // layout: SWIZZLE_64B
+    return d;
+}
+
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                          // D format fp32
