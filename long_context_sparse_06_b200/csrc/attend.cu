@@ -55,6 +55,8 @@ constexpr int kStageBytes = 9 * kBlk;         // 72 KB
 constexpr int kQBytes = 9 * (kH * 128);       // 72 KB
 constexpr int kAtThreads = 448;   // 4 softmax, 8 producers, 1 Q.K^T issuer, 1 P.V issuer
 constexpr int kWarpQK = 12, kWarpPV = 13;
+constexpr int kProdWarps = 8, kProdThreads = kProdWarps * 32;
+constexpr int kRowsPerWarp = kChunk / kProdWarps;   // gathered rows per producer warp and chunk
 constexpr size_t kAtSmem = 1024 + kQBytes + 2 * kStageBytes + kBlk;   // + the low part of P
 constexpr int kMaxSplits = 16;                // row-list splits per query (merged by attend_combine_kernel)
 constexpr int kOPitchF32 = kDv * 4 + 16;      // staged O rows (padded)
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         mbar_init(&bars.qfull, 1);
         for (int i = 0; i < 2; ++i) {
             for (int hf = 0; hf < 2; ++hf) {
-                mbar_init(&bars.kfull[i][hf], 128);   // the stage's four producer warps
+                mbar_init(&bars.kfull[i][hf], kProdThreads);   // every producer thread
                 mbar_init(&bars.kempty[i][hf], 1);
             }
             mbar_init(&bars.pfull[i], 128);
@@ -273,19 +275,21 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     };
 
     // ---- producers: warps 4-7 fill stage 0 (local chunks 0, 2, ...), warps 8-11 stage 1.
-    // A whole chunk of consecutive rows (window rows; HCA's compressed rows) comes by TMA,
-    // issued by the group's first thread: bf16 rows as one tile load per 128-byte column
-    // block; FP8 rows as their codes, which the group then widens to bf16 in shared memory.
-    // Other chunks are gathered row by row, warp pw of the group owning rows pw, pw+4, ...,
-    // pw+60 (lane i < 16 resolves row pw+4i): bf16 rows with 16-byte cp.async, FP8 rows
+    // All eight producer warps fill each chunk, chunks in order (a gather runs at about 60
+    // GB/s per SM from eight issuing warps, 39 from four).  A whole chunk of consecutive rows
+    // (window rows; HCA's compressed rows) comes by TMA, issued by the first producer thread:
+    // bf16 rows as one tile load per 128-byte column block; FP8 rows as their codes, which
+    // the producers then widen to bf16 in shared memory.  Other chunks are gathered row by
+    // row, warp pw owning rows pw, pw+8, ..., pw+56 (lane i < 8 resolves row pw+8i): bf16
+    // rows with 16-byte cp.async, FP8 rows
     // loaded, converted (exact with the power-of-two block scale) and stored.  The gathers
     // write zeros for rows past the chunk's valid count, so a partial chunk never reads
     // rows outside the query's row set (they may hold anything, NaN included).  All write
     // the SW128 layout both MMAs read.
     const bool producer = warp >= 4 && warp < 12;
-    const int pst = (warp - 4) >> 2, pw = (warp - 4) & 3;
+    const int pw = warp - 4;   // producer warp 0..7
     auto contiguous = [&](int64_t gc) { return (gc < nwc || sel == nullptr) && chunk_valid(gc) == kChunk; };
-    uint32_t raw_fills = 0;   // FP8 TMA fills of this group so far (rawfull parity)
+    uint32_t raw_par = 0;     // FP8 TMA fills: bit st = phase parity of rawfull[st]
     auto row_src = [&](int64_t gc, int rr) -> const uint8_t* {
         if (rr >= chunk_valid(gc)) return nullptr;
         if (gc < nwc)
@@ -295,90 +299,83 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         return static_cast<const uint8_t*>(a.comp) + (b * a.N_c + e) * row_bytes;
     };
     auto my_row_src = [&](int64_t gc) -> const uint8_t* {
-        return (lane < 16 && !contiguous(gc)) ? row_src(gc, pw + 4 * lane) : nullptr;
+        return (lane < kRowsPerWarp && !contiguous(gc)) ? row_src(gc, pw + kProdWarps * lane) : nullptr;
     };
-    // Fills stage pst with global chunk gc (its u-th use; u >= 1 waits for the P.V of the
+    // Fills stage st with global chunk gc (its u-th use; u >= 1 waits for the P.V of the
     // previous use to release the halves) and arrives on both halves' kfull (the TMA bytes
     // complete them).  Returns false when a wait ran out.
-    auto wait_half = [&](int u, int hf) -> bool {
-        return u < 1 || group_all(1 + pst, 128, mbar_wait(&bars.kempty[pst][hf], (uint32_t)((u - 1) & 1), status, 310 + hf));
+    auto wait_half = [&](int u, int hf, int st) -> bool {
+        return u < 1 ||
+               group_all(1, kProdThreads, mbar_wait(&bars.kempty[st][hf], (uint32_t)((u - 1) & 1), status, 310 + hf));
     };
-    auto fill = [&](int64_t gc, const uint8_t* my_src, int u) -> bool {
-        uint8_t* dst = stage_s + pst * kStageBytes;
+    auto fill = [&](int64_t gc, const uint8_t* my_src, int u, int st) -> bool {
+        uint8_t* dst = stage_s + st * kStageBytes;
         if (contiguous(gc) && !FP8) {
             // bf16 rows by TMA, half by half: the first half's load starts as soon as P.V has
             // released it
             const bool w = gc < nwc;
             const int row0 = w ? (int)(b * a.Tw + wp.win_lo + gc * kChunk) : (int)(b * a.N_c + (gc - nwc) * kChunk);
             for (int hf = 0; hf < 2; ++hf) {
-                if (!wait_half(u, hf)) return false;
+                if (!wait_half(u, hf, st)) return false;
                 const int b0 = hf ? kHalfBlocks : 0, b1 = hf ? 9 : kHalfBlocks;
                 if (pw == 0 && lane == 0) {
-                    mbar_arrive_expect_tx(&bars.kfull[pst][hf], (b1 - b0) * kBlk);
+                    mbar_arrive_expect_tx(&bars.kfull[st][hf], (b1 - b0) * kBlk);
                     for (int blk = b0; blk < b1; ++blk)
-                        tma_load_2d(dst + blk * kBlk, w ? &map_w : &map_c, &bars.kfull[pst][hf], blk * 64, row0);
+                        tma_load_2d(dst + blk * kBlk, w ? &map_w : &map_c, &bars.kfull[st][hf], blk * 64, row0);
                 } else {
-                    mbar_arrive(&bars.kfull[pst][hf]);
+                    mbar_arrive(&bars.kfull[st][hf]);
                 }
             }
             return true;
         }
         // every other fill writes the whole stage: wait for both halves first
-        if (!wait_half(u, 0) || !wait_half(u, 1)) return false;
+        if (!wait_half(u, 0, st) || !wait_half(u, 1, st)) return false;
         if (FP8 && contiguous(gc)) {
             const bool w = gc < nwc;
             const int row0 = w ? (int)(b * a.Tw + wp.win_lo + gc * kChunk) : (int)(b * a.N_c + (gc - nwc) * kChunk);
             {
                 // the codes of column block j (64 rows x 64 B) land in the upper half of
-                // block j, the RoPE dims (bf16, 128-byte swizzle) in block 8; thread tg then
-                // widens 16 codes of rows tg/4 and tg/4 + 32 per block (piece tg%4), reading
-                // block j+1's codes before the group barrier that lets block j+1 be written
+                // block j, the RoPE dims (bf16, 128-byte swizzle) in block 8; producer thread
+                // tg then widens 16 codes of row tg/4 per block (piece tg%4), reading block
+                // j+1's codes before the producers' barrier that lets block j+1 be written
                 const int tg = pw * 32 + lane;
                 if (tg == 0) {
-                    mbar_arrive_expect_tx(&bars.rawfull[pst], 8 * (kBlk / 2) + kBlk);
+                    mbar_arrive_expect_tx(&bars.rawfull[st], 8 * (kBlk / 2) + kBlk);
                     for (int j = 0; j < 8; ++j)
-                        tma_load_2d(dst + j * kBlk + kBlk / 2, w ? &map_w : &map_c, &bars.rawfull[pst], j * 64, row0);
-                    tma_load_2d(dst + 8 * kBlk, w ? &map_wr : &map_cr, &bars.rawfull[pst], 512, row0);
+                        tma_load_2d(dst + j * kBlk + kBlk / 2, w ? &map_w : &map_c, &bars.rawfull[st], j * 64, row0);
+                    tma_load_2d(dst + 8 * kBlk, w ? &map_wr : &map_cr, &bars.rawfull[st], 512, row0);
                 }
                 const int r1 = tg >> 2, piece = tg & 3;
                 const uint8_t* scales = static_cast<const uint8_t*>(w ? a.win : a.comp) + (int64_t)row0 * 656 + 640;
                 const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + (int64_t)r1 * 656));
-                const float4 s2 = __ldg(reinterpret_cast<const float4*>(scales + (int64_t)(r1 + 32) * 656));
-                const bool landed =
-                    group_all(1 + pst, 128, mbar_wait(&bars.rawfull[pst], raw_fills & 1u, status, 311));
-                ++raw_fills;
+                const bool landed = group_all(1, kProdThreads,
+                                              mbar_wait(&bars.rawfull[st], (raw_par >> st) & 1u, status, 311));
+                raw_par ^= 1u << st;
                 if (landed) {
                     const uint4* raw0 = reinterpret_cast<const uint4*>(dst + kBlk / 2);
-                    uint4 c1 = raw0[tg], c2 = raw0[tg + 128];
-                    group_bar(1 + pst, 128);
+                    uint4 c1 = raw0[tg];
+                    group_bar(1, kProdThreads);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        uint4 n1 = c1, n2 = c2;
-                        if (j < 7) {
-                            const uint4* rawn = reinterpret_cast<const uint4*>(dst + (j + 1) * kBlk + kBlk / 2);
-                            n1 = rawn[tg];
-                            n2 = rawn[tg + 128];
-                        }
+                        uint4 n1 = c1;
+                        if (j < 7) n1 = reinterpret_cast<const uint4*>(dst + (j + 1) * kBlk + kBlk / 2)[tg];
                         const int sj = j >> 1;
                         const float f1 = sj == 0 ? s1.x : sj == 1 ? s1.y : sj == 2 ? s1.z : s1.w;
-                        const float f2 = sj == 0 ? s2.x : sj == 1 ? s2.y : sj == 2 ? s2.z : s2.w;
                         widen_piece(dst + j * kBlk, r1, 2 * piece, c1, f1);
-                        widen_piece(dst + j * kBlk, r1 + 32, 2 * piece, c2, f2);
-                        if (j < 7) group_bar(1 + pst, 128);
+                        if (j < 7) group_bar(1, kProdThreads);
                         c1 = n1;
-                        c2 = n2;
                     }
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&bars.kfull[pst][0]);
-                mbar_arrive(&bars.kfull[pst][1]);
+                mbar_arrive(&bars.kfull[st][0]);
+                mbar_arrive(&bars.kfull[st][1]);
                 return true;
             }
         }
         if constexpr (!FP8) {
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const int rr = pw + 4 * i;
+#pragma unroll
+            for (int i = 0; i < kRowsPerWarp; ++i) {
+                const int rr = pw + kProdWarps * i;
                 const uint8_t* src = reinterpret_cast<const uint8_t*>(
                     __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), i));
                 const bool valid = src != nullptr;
@@ -390,8 +387,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             cp_async_wait<0>();
         } else {
             // FP8 row: 32 content pieces of 16 codes (-> 32 bf16) and 8 RoPE pieces of 8 bf16;
-            // 8 rows' loads in flight per lane
-            for (int i0 = 0; i0 < 16; i0 += 8) {
+            // the warp's 8 rows' loads in flight per lane
+            for (int i0 = 0; i0 < kRowsPerWarp; i0 += 8) {
                 uint4 cv[8], rv[8];
                 float sc[8];
 #pragma unroll
@@ -409,7 +406,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int rr = pw + 4 * (i0 + u);
+                    const int rr = pw + kProdWarps * (i0 + u);
                     // lane's 16 codes are the row's chunks 2*lane, 2*lane+1: block lane/4
                     widen_piece(dst + (lane >> 2) * kBlk, rr, (lane & 3) * 2, cv[u], sc[u]);
                     if (lane < 8) *reinterpret_cast<uint4*>(dst + 8 * kBlk + sw128_off(rr, lane)) = rv[u];
@@ -417,20 +414,15 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&bars.kfull[pst][0]);
-        mbar_arrive(&bars.kfull[pst][1]);
+        mbar_arrive(&bars.kfull[st][0]);
+        mbar_arrive(&bars.kfull[st][1]);
         return true;
     };
-    // Window chunks need no selection: the first chunk of each stage is filled before the
-    // wait for the preceding kernel when it is a window chunk of this split.
-    bool pre = false;
-    if (producer) {
-        const int64_t gc = gcof(pst);
-        if (gc < nwc) {
-            fill(gc, my_row_src(gc), 0);
-            pre = true;
-        }
-    }
+    // Window chunks need no selection: the producers fill them (up to both stages) before
+    // the wait for the preceding kernel.
+    int pre = 0;   // local chunks filled before the wait
+    if (producer)
+        while (pre < 2 && gcof(pre) < nwc && fill(gcof(pre), my_row_src(gcof(pre)), 0, pre)) ++pre;
 #if defined(__CUDA_ARCH__)
     asm volatile("griddepcontrol.wait;" ::: "memory");
 #endif
@@ -522,16 +514,15 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             mma_commit(&bars.odone);
         }
     } else if (producer) {
-        // ---------------- producer loop (the group's chunks pst, pst+2, ...); a stage is
-        // refilled once the P.V that read it is complete.  The next chunk's row sources are
-        // resolved while this chunk's copies are in flight.
-        const uint8_t* nxt = (pst < nch) ? my_row_src(gcof(pst)) : nullptr;
-        for (int c = pst; c < nch; c += 2) {
+        // ---------------- producer loop: local chunks pre, pre+1, ... in order, stage c & 1;
+        // a stage is refilled once the P.V that read it is complete.  The next chunk's row
+        // sources are resolved while this chunk's copies are in flight.
+        const uint8_t* nxt = (pre < nch) ? my_row_src(gcof(pre)) : nullptr;
+        for (int c = pre; c < nch; ++c) {
             const uint8_t* my_src = nxt;
-            const int u = c >> 1;
-            if (c + 2 < nch) nxt = my_row_src(gcof(c + 2));
-            // the group leaves together (its waits are group decisions)
-            if (!(pre && c == pst) && !fill(gcof(c), my_src, u)) break;
+            if (c + 1 < nch) nxt = my_row_src(gcof(c + 1));
+            // the producers leave together (their waits are group decisions)
+            if (!fill(gcof(c), my_src, c >> 1, c & 1)) break;
         }
     } else if (warp < 4) {
         // ---------------- softmax / correction / epilogue: warps 0..3.  Warp q owns heads
