@@ -328,6 +328,34 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
             return true;
         }
+        if constexpr (!FP8) {
+            // gathered bf16 rows, half by half like the TMA fills: column blocks 0-3 (lane l
+            // copies 16-byte chunk l of each of the warp's rows) as soon as P.V has released
+            // them, then blocks 4-8; each half is announced once its copies have landed
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                if (!wait_half(u, hf, st)) return false;
+#pragma unroll
+                for (int i = 0; i < kRowsPerWarp; ++i) {
+                    const int rr = pw + kProdWarps * i;
+                    const uint8_t* src = reinterpret_cast<const uint8_t*>(
+                        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), i));
+                    const bool valid = src != nullptr;
+                    const uint8_t* base = valid ? src : static_cast<const uint8_t*>(a.comp);
+                    for (int ch = hf ? 32 + lane : lane; ch < (hf ? 72 : 32); ch += 32)
+                        cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), base + (valid ? ch * 16 : 0),
+                                    valid);
+                }
+                cp_async_commit();
+            }
+            cp_async_wait<1>();
+            fence_proxy_async_smem();
+            mbar_arrive(&bars.kfull[st][0]);
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&bars.kfull[st][1]);
+            return true;
+        }
         // every other fill writes the whole stage: wait for both halves first
         if (!wait_half(u, 0, st) || !wait_half(u, 1, st)) return false;
         if (FP8 && contiguous(gc)) {
@@ -372,20 +400,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 return true;
             }
         }
-        if constexpr (!FP8) {
-#pragma unroll
-            for (int i = 0; i < kRowsPerWarp; ++i) {
-                const int rr = pw + kProdWarps * i;
-                const uint8_t* src = reinterpret_cast<const uint8_t*>(
-                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), i));
-                const bool valid = src != nullptr;
-                const uint8_t* base = valid ? src : static_cast<const uint8_t*>(a.comp);
-                for (int ch = lane; ch < 72; ch += 32)
-                    cp_async_16(dst + (ch >> 3) * kBlk + sw128_off(rr, ch & 7), base + (valid ? ch * 16 : 0), valid);
-            }
-            cp_async_commit();
-            cp_async_wait<0>();
-        } else {
+        {
             // FP8 row: 32 content pieces of 16 codes (-> 32 bf16) and 8 RoPE pieces of 8 bf16;
             // the warp's 8 rows' loads in flight per lane
             for (int i0 = 0; i0 < kRowsPerWarp; i0 += 8) {
