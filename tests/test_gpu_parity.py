@@ -655,6 +655,30 @@ def test_index_fp4_bit_exact(L, orc):
         np.testing.assert_array_equal(idx[b, 0], orc.topk(ref.astype(np.float32), k))
 
 
+@pytest.mark.parametrize("B,Q,Nc", [(2, 9, 1000), (3, 40, 130)])
+def test_index_fp4_causal_groups(L, orc, B, Q, Nc):
+    """FP4 index over several queries per request with causal availability: query groups
+    change often (the per-group scale factors), tiles past a query's available entries are
+    skipped by every role of the kernel alike, the last tile is ragged, and one query has no
+    available entry.  Scores of the available entries and the selection bit-exact."""
+    H, k = 64, 64
+    qI = randn(f"g.i4c.q{Q}", (B, Q, H, 128), dtype=torch.bfloat16)
+    w = randn(f"g.i4c.w{Q}", (B, Q, H), std=1 / 8)
+    planes, kp, ks = _fp4_keys(L, orc, f"g.i4c.k{Q}", B, Nc)
+    q_pos = (torch.arange(Q, dtype=torch.int64) * (4 * Nc // Q + 9) - 1).reshape(1, Q).repeat(B, 1)
+    q_pos[:, 0] = 0                                   # n_avail = 0
+    q_pos[B - 1] += 6
+    idx, sc = L.csa_index_topk(qI.to(DEV), w.to(DEV), planes, k, q_pos=q_pos.to(DEV), m=4, N_c=Nc,
+                               kI_dtype=L.FP4, want_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.float().cpu().numpy()
+    for b in range(B):
+        for q in range(Q):
+            n = orc.n_avail(int(q_pos[b, q]), 4, Nc)
+            ref = orc.index_scores_fp4(qI[b, q].float().numpy(), w[b, q].numpy(), kp[b, :n], ks[b, :n])
+            np.testing.assert_array_equal(sc[b, q, :n], ref, err_msg=f"b {b} q {q}")
+            np.testing.assert_array_equal(idx[b, q], orc.topk(ref.astype(np.float32), k), err_msg=f"b {b} q {q}")
+
+
 def test_decode_fused_mixed_precision(L, orc):
     """The 1M-context config's formats at a small size: FP8 KV with bf16 RoPE dims,
     FP4 index keys, bf16 scores, k = 1024."""
