@@ -16,7 +16,10 @@
 //    [64 x 128] into one of two slots; warp 1 issues tcgen05.mma (M = 128 keys,
 //    N = 64 heads, K = 128) into one of four TMEM accumulators; warps 2-5 read
 //    the accumulator rows (one key per thread) with tcgen05.ld and apply the
-//    ReLU / weighted head sum in fp32, writing one score per key.
+//    ReLU / weighted head sum in fp32, writing one score per key.  The prefill form
+//    (four queries per group, N = 256, two accumulators) has a second epilogue group,
+//    warps 6-9: the groups take alternate work items, one accumulator each, since the
+//    head chains of four queries take longer than the MMA of an item.
 #include <utility>
 
 #include "lcs_common.cuh"
@@ -69,9 +72,10 @@ constexpr int kBM = 128;        // keys per tile (MMA M)
 constexpr int kHeads = 64;      // index heads per query
 constexpr int kDI = 128;        // index dim (MMA K)
 constexpr int kATile = kBM * kDI * 2;        // 32 KB
-constexpr int kIxThreads = 192;
 template <int QB>
 struct IxCfg {
+    static constexpr int kEpiGroups = QB == 1 ? 1 : 2;     // epilogue groups of four warps
+    static constexpr int kThreads = 64 + 128 * kEpiGroups;
     static constexpr int kN = kHeads * QB;                 // MMA N
     static constexpr int kStages = QB == 1 ? 4 : 3;
     static constexpr int kAcc = QB == 1 ? 4 : 2;
@@ -106,7 +110,7 @@ __device__ __forceinline__ int64_t group_avail(const int64_t* q_pos, int64_t b, 
 }
 
 template <int QB>
-__global__ void __launch_bounds__(kIxThreads, 1)
+__global__ void __launch_bounds__(IxCfg<QB>::kThreads, 1)
     index_bf16_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                          const float* __restrict__ w, int64_t Q, int64_t N_c, const int64_t* __restrict__ q_pos,
                          int m, int64_t n_groups, float* __restrict__ scores, int* status) {
@@ -224,11 +228,13 @@ __global__ void __launch_bounds__(kIxThreads, 1)
             if (prev_g >= 0) mma_commit(&bars.bempty[slot]);
         }
     } else {
-        // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4, thread = key.
-        // The QB queries' head chains run interleaved (each in its own fixed order h = 0..63),
-        // so that their fused multiply-adds hide one another's latency.
+        // ---------------- epilogue: warps 2..5 (and 6..9, the second group, which takes the
+        // odd work items); TMEM lane quarter = warp % 4, thread = key.  The QB queries' head
+        // chains run interleaved (each in its own fixed order h = 0..63), so that their
+        // fused multiply-adds hide one another's latency.
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
+        const int egroup = (warp - 2) >> 2;
         int64_t n_it = 0, av_g = -1, av_n = 0;
         int64_t nq[QB];
         const float4* wq[QB];
@@ -248,6 +254,10 @@ __global__ void __launch_bounds__(kIxThreads, 1)
                 }
             }
             if (tile * kBM >= av_n) continue;
+            if (C::kEpiGroups > 1 && (int)(n_it % C::kEpiGroups) != egroup) {   // the other group's item
+                ++n_it;
+                continue;
+            }
             const int ac = (int)(n_it % C::kAcc);
             if (!mbar_wait(&bars.afull[ac], (uint32_t)((n_it / C::kAcc) & 1), status, 106)) break;
             tc_fence_after();
@@ -333,12 +343,12 @@ cudaError_t launch_index_bf16_tc(const void* qI, const float* w, const void* kI,
     if (batched) {
         cudaError_t e = set_smem_once(reinterpret_cast<const void*>(index_bf16_tc_kernel<4>), IxCfg<4>::kSmem);
         if (e != cudaSuccess) return e;
-        return launch_k(index_bf16_tc_kernel<4>, dim3((unsigned)grid), dim3(kIxThreads), IxCfg<4>::kSmem, s, pdl, mk,
+        return launch_k(index_bf16_tc_kernel<4>, dim3((unsigned)grid), dim3(IxCfg<4>::kThreads), IxCfg<4>::kSmem, s, pdl, mk,
                         mq, w, Q, N_c, q_pos, m, n_groups, scores, status);
     }
     cudaError_t e = set_smem_once(reinterpret_cast<const void*>(index_bf16_tc_kernel<1>), IxCfg<1>::kSmem);
     if (e != cudaSuccess) return e;
-    return launch_k(index_bf16_tc_kernel<1>, dim3((unsigned)grid), dim3(kIxThreads), IxCfg<1>::kSmem, s, pdl, mk, mq,
+    return launch_k(index_bf16_tc_kernel<1>, dim3((unsigned)grid), dim3(IxCfg<1>::kThreads), IxCfg<1>::kSmem, s, pdl, mk, mq,
                     w, Q, N_c, q_pos, m, n_groups, scores, status);
 }
 
