@@ -11,13 +11,19 @@ least 300 tokens.  Checks:
   * FP8 KV rows and FP4 index keys: the stored bytes are exactly the library's cache
     writers (pinned bit-exact to the oracle's quantisers) applied to the fp32 entries;
   * bf16 inputs and storage: within 1e-4 of CacheState on the bf16 inputs with fp32
-    storage, and the bf16 caches are exactly those values rounded.
+    storage, and the bf16 caches are exactly those values rounded;
+  * the decode loop: a fused CSA decode step (k covering the whole compressed cache) and a
+    fused HCA decode step run directly on the appended bf16 caches, against the oracle's
+    attention over CacheState's entries (rounded to bf16, unwritten slots zero), within
+    2e-2 x RMS.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
 
-from helpers import assert_close_abs
+from helpers import assert_close_abs, assert_close_rel_rms, randn
 
 pytestmark = pytest.mark.gpu
 
@@ -131,3 +137,34 @@ def test_cache_update_stream(L, orc):
     gb16 = _stream(L, inp, torch.bfloat16, "bf16", "bf16", "bf16")
     for k in ("comp", "kI", "hca", "win"):
         assert torch.equal(gb16[k], gb32[k].to(torch.bfloat16)), k
+
+
+def test_decode_on_appended_caches(L, orc):
+    inp = _inputs()
+    g = _stream(L, inp, torch.bfloat16, "bf16", "bf16", "bf16")
+    sts = _oracle_states(orc, inp, True)
+    bf = torch.bfloat16
+    scale = 1 / math.sqrt(D)
+    q = randn("cu.dq", (B, 64, D), dtype=bf)
+    qI = randn("cu.dqi", (B, 64, DI), dtype=bf)
+    w = randn("cu.dw", (B, 64), std=1 / 8)
+    idx = torch.empty((B, NC), dtype=torch.int32, device=DEV)
+    out_c = L.decode_fused(L.MODE_CSA, q.to(DEV), g["comp"], g["win"], 512, scale, qI=qI.to(DEV), w=w.to(DEV),
+                           kI=g["kI"], k=NC, idx_out=idx, out_dtype=torch.float32).cpu().numpy()
+    out_h = L.decode_fused(L.MODE_HCA, q.to(DEV), g["hca"], g["win"], 512, scale,
+                           out_dtype=torch.float32).cpu().numpy()
+    assert torch.equal(idx.cpu(), torch.arange(NC, dtype=torch.int32).repeat(B, 1))   # k covers every slot
+    r16 = lambda a: torch.from_numpy(np.asarray(a, np.float64)).to(bf).double().numpy()   # noqa: E731
+    for b, cs in enumerate(sts):
+        comp_o = np.zeros((NC, D))
+        comp_o[:len(cs.csa)] = r16(cs.csa)
+        hca_o = np.zeros((NH, D))
+        hca_o[:len(cs.hca)] = r16(cs.hca)
+        win_o = np.zeros((128, D))
+        for p, rowv in cs.window:
+            win_o[p % 128] = r16(rowv)
+        qb = q[b].double().numpy()
+        o, _ = orc.csa_attend(qb, comp_o, np.arange(NC, dtype=np.int32), win_o, 0, -1, 128, 512, scale)
+        assert_close_rel_rms(out_c[b], o, 2e-2, f"CSA decode on the appended caches b{b}")
+        o, _ = orc.csa_attend(qb, hca_o, np.arange(NH, dtype=np.int32), win_o, 0, -1, 128, 512, scale)
+        assert_close_rel_rms(out_h[b], o, 2e-2, f"HCA decode on the appended caches b{b}")
