@@ -12,17 +12,18 @@
 //
 // Few rows of at most 65536 entries (decode over 128K tokens, the tiny prefill): a cluster
 // of up to 8 CTAs per row with the whole row in registers and an exact radix select
-// (topk_row_kernel, below).  Longer rows: one CTA of 512 threads per query row, or a
-// cluster of them per row when there are few rows:
+// (topk_row_kernel, below).  Longer rows: one CTA of 256 threads per query row, two CTAs
+// per SM, or a cluster of 512-thread CTAs per row when there are few rows:
 //  1. Lower bound: a fixed strided sample of 512 keys is histogrammed over the
-//     top 14 key bits (sign, exponent, top mantissa bits); the lower edge of the
+//     top 13 (256 threads) or 14 (512 threads) key bits (sign, exponent, top
+//     mantissa bits); the lower edge of the
 //     bin holding the sample's rank-r element, r about 1.5 k x sample/row + 8,
 //     bounds the k-th score from below with overwhelming probability.
 //  2. One pass over the row: each lane loads 32 consecutive keys with 16-byte
 //     vector loads and appends those >= the bound to its warp's buffer; slots
 //     come from per-lane counts and a warp scan, so candidates stay in index
 //     order.
-//  3. The candidates (about 1.5 k) are histogrammed on the same 14 bits; a
+//  3. The candidates (about 1.5 k) are histogrammed on the same bits; a
 //     suffix scan finds the bin holding the k-th largest; that bin's members are
 //     ranked exactly by counting on the composite key; an ordered compaction over
 //     the candidate list (warp slices, __ballot_sync / __popc for the slots) writes
@@ -32,6 +33,7 @@
 // row falls back to an exact MSB-first radix select (8-bit digits) followed by
 // an ordered ballot compaction.  Nothing depends on the order of the atomics,
 // so every step is deterministic.
+#include <mutex>
 #include <utility>
 
 #include "lcs_common.cuh"
@@ -41,25 +43,35 @@ namespace lcs {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kBinBits = 14;
-constexpr int kBins = 1 << kBinBits;
-constexpr int kCandCap = 2048;                 // threshold-bin elements ranked by counting
-constexpr int kWarpCap = 512;                  // per-warp candidate buffer
-constexpr int kListCap = kWarps * kWarpCap;    // all candidates
-constexpr int kMaxP = 16;                      // CTAs per row (one cluster)
-static_assert(kMaxP <= kWarps, "per-rank counts reuse the per-warp arrays");
+// Block shapes of topk_kernel: 512 threads when a row is split over a cluster (few long
+// rows), 256 threads when each row has a CTA of its own (many rows: prefill), two CTAs per
+// SM, so that one row's passes run while the other's wait at block barriers.
+template <int NT>
+struct TkCfg {
+    static constexpr int kThreads = NT;
+    static constexpr int kWarps = NT / 32;
+    static constexpr int kBinBits = NT >= 512 ? 14 : 13;
+    static constexpr int kBins = 1 << kBinBits;
+    static constexpr int kWarpCap = 512;                   // per-warp candidate buffer
+    static constexpr int kListCap = kWarps * kWarpCap;     // all candidates
+    static_assert(kWarps <= 32, "one warp scans the per-warp sums");
+};
+constexpr int kCandCap = 2048;    // threshold-bin elements ranked by counting
+constexpr int kSamples = 512;     // keys in the sampled lower bound
+constexpr int kMaxP = 16;         // CTAs per row (one cluster of 512-thread CTAs)
+static_assert(kMaxP <= TkCfg<512>::kWarps, "per-rank counts reuse the per-warp arrays");
 
+template <int NT>
 struct TopkSmem {
-    uint32_t bins[kBins + kBins / 32];          // 64 KB histogram, one pad word per 32 bins
-    unsigned long long wbuf[kListCap];          // per-warp candidate buffers (64 KB)
-    unsigned long long list[kListCap];          // compacted candidates, index order (64 KB)
-    uint8_t take[kListCap];                     // candidate selected?
+    using C = TkCfg<NT>;
+    uint32_t bins[C::kBins + C::kBins / 32];    // histogram, one pad word per 32 bins
+    unsigned long long wbuf[C::kListCap];       // per-warp candidate buffers
+    unsigned long long list[C::kListCap];       // compacted candidates, index order
+    uint8_t take[C::kListCap];                  // candidate selected?
     uint16_t mpos[kCandCap];                    // list positions of the threshold bin's members
     uint32_t hist[256], scan[256];              // radix fallback
-    uint32_t warp_cnt[kWarps], warp_off[kWarps], warp_gt[kWarps], warp_sel[kWarps];
-    uint32_t wsum[kWarps];
+    uint32_t warp_cnt[C::kWarps], warp_off[C::kWarps], warp_gt[C::kWarps], warp_sel[C::kWarps];
+    uint32_t wsum[C::kWarps];
     uint32_t digit, krem, tbin, above, fail, total;
 };
 
@@ -74,7 +86,9 @@ __device__ __forceinline__ uint32_t load_key(const void* row, int64_t i) {
 }
 
 // ---------------------------------------------------------- exact fallback
-__device__ void pick_digit(TopkSmem& sm) {
+template <int NT>
+__device__ void pick_digit(TopkSmem<NT>& sm) {
+    static_assert(NT >= 256, "one thread per digit");
     const int t = threadIdx.x;
     if (t < 256) sm.scan[t] = sm.hist[255 - t];
     __syncthreads();
@@ -93,9 +107,10 @@ __device__ void pick_digit(TopkSmem& sm) {
     __syncthreads();
 }
 
-template <bool BF16>
-__device__ void radix_select(TopkSmem& sm, const void* srow, int64_t n, int k, int32_t* out) {
+template <bool BF16, int NT>
+__device__ void radix_select(TopkSmem<NT>& sm, const void* srow, int64_t n, int k, int32_t* out) {
     constexpr int kBits = BF16 ? 16 : 32;
+    constexpr int kThreads = NT, kWarps = NT / 32;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     if (t == 0) sm.krem = (uint32_t)k;
     uint32_t prefix = 0;
@@ -146,8 +161,9 @@ __device__ void radix_select(TopkSmem& sm, const void* srow, int64_t n, int k, i
 
 // Exclusive prefix over the kWarps per-warp values in sm.wsum (scanned in place by
 // warp 0; lanes >= kWarps carry zeros and write nothing).
-static_assert(kWarps <= 32, "one warp scans the per-warp sums");
-__device__ __forceinline__ void scan_warp_sums(TopkSmem& sm) {
+template <int NT>
+__device__ __forceinline__ void scan_warp_sums(TopkSmem<NT>& sm) {
+    constexpr int kWarps = NT / 32;
     if (threadIdx.x < 32) {
         const uint32_t v = (threadIdx.x < kWarps) ? sm.wsum[threadIdx.x] : 0u;
         uint32_t incl = v;
@@ -164,9 +180,11 @@ __device__ __forceinline__ void scan_warp_sums(TopkSmem& sm) {
 
 // Block-wide: the bin holding the k-th largest of the histogram (bins in descending
 // order of value from the top).  Sets sm.tbin and sm.above (count in higher bins).
-__device__ void find_bin(TopkSmem& sm, uint32_t k) {
+template <int NT>
+__device__ void find_bin(TopkSmem<NT>& sm, uint32_t k) {
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    constexpr int kPer = kBins / kThreads;      // thread 0 owns the top bins
+    constexpr int kBins = TkCfg<NT>::kBins;
+    constexpr int kPer = kBins / NT;            // thread 0 owns the top bins
     const int hi_bin = kBins - 1 - t * kPer;
     uint32_t c[kPer];
     uint32_t local = 0;
@@ -252,13 +270,17 @@ __device__ __forceinline__ void batch_keys(const char* srow, int64_t bb, int64_t
     }
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restrict__ scores, int64_t N_c,
-                                                           const int64_t* __restrict__ q_pos, int m, int k,
-                                                           int32_t* __restrict__ idx_out, int P) {
+// NT = 512: one CTA per SM, P CTAs per row in a cluster.  NT = 256: P = 1, two CTAs per SM.
+template <bool BF16, int NT>
+__global__ void __launch_bounds__(NT, 512 / NT) topk_kernel(const void* __restrict__ scores, int64_t N_c,
+                                                            const int64_t* __restrict__ q_pos, int m, int k,
+                                                            int32_t* __restrict__ idx_out, int P) {
+    using Cfg = TkCfg<NT>;
+    constexpr int kThreads = NT, kWarps = Cfg::kWarps, kBins = Cfg::kBins;
+    constexpr int kWarpCap = Cfg::kWarpCap, kListCap = Cfg::kListCap;
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
-    constexpr int kShift = (BF16 ? 16 : 32) - kBinBits;
+    TopkSmem<NT>& sm = *reinterpret_cast<TopkSmem<NT>*>(smem_raw);
+    constexpr int kShift = (BF16 ? 16 : 32) - Cfg::kBinBits;
     const int64_t row = blockIdx.x / P;
     const int rank = (int)(blockIdx.x - row * P);   // == rank in the row's cluster
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -287,10 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
     __syncthreads();
     uint32_t T = 0;
     if (n > kListCap / 2) {
-        atomicAdd(&sm.bins[hb(load_key<BF16>(srow, (int64_t)(((uint64_t)t * (uint64_t)n) / kThreads)) >> kShift)], 1u);
+#pragma unroll
+        for (int j = 0; j < kSamples / kThreads; ++j) {   // sample s = t + j * kThreads at s * n / kSamples
+            const uint64_t s = (uint64_t)(t + j * kThreads);
+            atomicAdd(&sm.bins[hb(load_key<BF16>(srow, (int64_t)((s * (uint64_t)n) / kSamples)) >> kShift)], 1u);
+        }
         __syncthreads();
-        uint32_t r = (uint32_t)((3 * (int64_t)k * kThreads) / (2 * n)) + 8;
-        if (r > (uint32_t)kThreads) r = kThreads;
+        uint32_t r = (uint32_t)((3 * (int64_t)k * kSamples) / (2 * n)) + 8;
+        if (r > (uint32_t)kSamples) r = kSamples;
         find_bin(sm, r);
         T = sm.tbin << kShift;
         for (int i = t; i < kBins + kBins / 32; i += kThreads) sm.bins[i] = 0;
@@ -373,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const void* __restric
         for (uint32_t j = lane; j < wcnt; j += 32) sm.list[o + j] = wb[j];
     }
     __syncthreads();
-    if (P > 1) {
+    if constexpr (kWarps >= kMaxP) if (P > 1) {
         // ---- the row's CTAs form one cluster: CTA 0 appends the peers' candidate lists
         // (slices in rank order, so the list stays in index order) through distributed
         // shared memory, then selects; a missed bound falls back to CTA 0 alone.
@@ -787,15 +813,15 @@ int choose_ranks(int64_t rows, int64_t N_c) {
     static std::mutex mu;
     static int cache[kMaxP + 1];
     std::lock_guard<std::mutex> lock(mu);
-    const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16>);
+    const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16, 512>);
     for (; p > 1; --p) {
         if (cache[p] == 0) {
             int n = 0;
             if (p <= 8 || cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
                 cudaLaunchConfig_t cfg = {};
                 cfg.gridDim = dim3((unsigned)p);
-                cfg.blockDim = dim3(kThreads);
-                cfg.dynamicSmemBytes = sizeof(TopkSmem);
+                cfg.blockDim = dim3(512);
+                cfg.dynamicSmemBytes = sizeof(TopkSmem<512>);
                 cudaLaunchAttribute attr[1];
                 attr[0].id = cudaLaunchAttributeClusterDimension;
                 attr[0].val.clusterDim.x = (unsigned)p;
@@ -811,6 +837,42 @@ int choose_ranks(int64_t rows, int64_t N_c) {
         if (cache[p] >= rows) break;
     }
     return (int)(p < 1 ? 1 : p);
+}
+
+// topk_kernel<BF16, NT> over rows x P CTAs, P CTAs per row in one cluster.
+template <bool BF16, int NT>
+cudaError_t launch_topk_cta(const void* scores, int64_t rows, int64_t N_c, const int64_t* q_pos, int m, int k,
+                            int32_t* idx, cudaStream_t s, bool pdl, int P) {
+    const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16, NT>);
+    cudaError_t e = set_smem_once(kern, sizeof(TopkSmem<NT>));
+    if (e != cudaSuccess) return e;
+    if constexpr (NT < 512) {   // two CTAs per SM need the whole carveout as shared memory
+        static std::once_flag once;
+        std::call_once(once, [&] { e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100); });
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * P));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = sizeof(TopkSmem<NT>);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (P > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)P;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, topk_kernel<BF16, NT>, scores, N_c, q_pos, m, k, idx, P);
 }
 
 template <bool BF16>
@@ -845,30 +907,9 @@ cudaError_t launch_topk_t(const void* scores, int64_t rows, int64_t N_c, const i
         cfg.numAttrs = na;
         return cudaLaunchKernelEx(&cfg, topk_row_kernel<BF16>, scores, N_c, q_pos, m, k, idx, P);
     }
-    const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16>);
-    cudaError_t e = set_smem_once(kern, sizeof(TopkSmem));
-    if (e != cudaSuccess) return e;
     const int P = choose_ranks<BF16>(rows, N_c);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rows * P));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = sizeof(TopkSmem);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    int na = 0;
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = (unsigned)P;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    ++na;
-    if (pdl) {
-        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, topk_kernel<BF16>, scores, N_c, q_pos, m, k, idx, P);
+    if (P == 1) return launch_topk_cta<BF16, 256>(scores, rows, N_c, q_pos, m, k, idx, s, pdl, 1);
+    return launch_topk_cta<BF16, 512>(scores, rows, N_c, q_pos, m, k, idx, s, pdl, P);
 }
 }  // namespace
 
