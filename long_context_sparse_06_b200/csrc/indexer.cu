@@ -75,6 +75,8 @@ constexpr int kATile = kBM * kDI * 2;        // 32 KB
 template <int QB>
 struct IxCfg {
     static constexpr int kEpiGroups = QB == 1 ? 1 : 2;     // epilogue groups of four warps
+    static constexpr int kQG = QB / kEpiGroups;            // queries per epilogue group
+    static constexpr int kHStep = QB == 1 ? 16 : 32;       // heads per TMEM load round
     static constexpr int kThreads = 64 + 128 * kEpiGroups;
     static constexpr int kN = kHeads * QB;                 // MMA N
     static constexpr int kStages = QB == 1 ? 4 : 3;
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(IxCfg<QB>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kStages; ++i) { mbar_init(&bars.full[i], 1); mbar_init(&bars.empty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&bars.bfull[i], 1); mbar_init(&bars.bempty[i], 1); }
-        for (int i = 0; i < C::kAcc; ++i) { mbar_init(&bars.afull[i], 1); mbar_init(&bars.aempty[i], 4); }
+        for (int i = 0; i < C::kAcc; ++i) { mbar_init(&bars.afull[i], 1); mbar_init(&bars.aempty[i], 4 * C::kEpiGroups); }
         fence_barrier_init();
         prefetch_tmap(&map_k);
         prefetch_tmap(&map_q);
@@ -228,58 +230,59 @@ __global__ void __launch_bounds__(IxCfg<QB>::kThreads, 1)
             if (prev_g >= 0) mma_commit(&bars.bempty[slot]);
         }
     } else {
-        // ---------------- epilogue: warps 2..5 (and 6..9, the second group, which takes the
-        // odd work items); TMEM lane quarter = warp % 4, thread = key.  The QB queries' head
-        // chains run interleaved (each in its own fixed order h = 0..63), so that their
-        // fused multiply-adds hide one another's latency.
+        // ---------------- epilogue: warps 2..5 (and 6..9, the second group); TMEM lane
+        // quarter = warp % 4, thread = key.  Every group takes every work item, group e the
+        // queries e * kQG ... of the QB, so that an item's accumulator is released after
+        // half the head chains a thread would otherwise run.  A thread's kQG head chains run
+        // interleaved (each in its own fixed order h = 0..63), so that their fused
+        // multiply-adds hide one another's latency.
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int egroup = (warp - 2) >> 2;
+        const int q0 = egroup * C::kQG;
         int64_t n_it = 0, av_g = -1, av_n = 0;
-        int64_t nq[QB];
-        const float4* wq[QB];
+        int64_t nq[C::kQG];
+        const float4* wq[C::kQG];
         TileIt ti(it0, (int)tiles_per, (int)nqb);
         for (int64_t it = it0; it < it1; ++it, ti.next((int)tiles_per, (int)nqb)) {
             const int64_t tile = ti.tile;
             if (ti.g != av_g) {   // the group's queries: availability and head weights
                 av_g = ti.g;
-                av_n = 0;
+                av_n = group_avail<QB>(q_pos, ti.b, ti.q, Q, m, N_c);
 #pragma unroll
-                for (int qi = 0; qi < QB; ++qi) {
-                    const int64_t q = ti.q * QB + qi;
+                for (int qi = 0; qi < C::kQG; ++qi) {
+                    const int64_t q = ti.q * QB + q0 + qi;
                     const int64_t gq = ti.b * Q + (q < Q ? q : ti.q * QB);
                     nq[qi] = q < Q ? avail(q_pos, gq, m, N_c) : -1;
-                    av_n = nq[qi] > av_n ? nq[qi] : av_n;
                     wq[qi] = reinterpret_cast<const float4*>(w + gq * kHeads);   // L1-resident
                 }
             }
             if (tile * kBM >= av_n) continue;
-            if (C::kEpiGroups > 1 && (int)(n_it % C::kEpiGroups) != egroup) {   // the other group's item
-                ++n_it;
-                continue;
-            }
             const int ac = (int)(n_it % C::kAcc);
             if (!mbar_wait(&bars.afull[ac], (uint32_t)((n_it / C::kAcc) & 1), status, 106)) break;
             tc_fence_after();
-            float acc[QB];
+            float acc[C::kQG];
 #pragma unroll
-            for (int qi = 0; qi < QB; ++qi) acc[qi] = 0.f;
+            for (int qi = 0; qi < C::kQG; ++qi) acc[qi] = 0.f;
 #pragma unroll 1
-            for (int h0 = 0; h0 < kHeads; h0 += 16) {
-                uint32_t d[QB][16];
+            for (int h0 = 0; h0 < kHeads; h0 += C::kHStep) {
+                uint32_t d[C::kQG][C::kHStep];
 #pragma unroll
-                for (int qi = 0; qi < QB; ++qi)
-                    tmem_ld16(tmem_addr(tmem, quarter * 32, ac * C::kN + qi * kHeads + h0), d[qi]);
+                for (int qi = 0; qi < C::kQG; ++qi) {
+                    const uint32_t ta = tmem_addr(tmem, quarter * 32, ac * C::kN + (q0 + qi) * kHeads + h0);
+                    if constexpr (C::kHStep == 32) tmem_ld32(ta, d[qi]);
+                    else tmem_ld16(ta, d[qi]);
+                }
                 tmem_ld_wait();
 #pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4) {
-                    float4 wv[QB];
+                for (int j4 = 0; j4 < C::kHStep / 4; ++j4) {
+                    float4 wv[C::kQG];
 #pragma unroll
-                    for (int qi = 0; qi < QB; ++qi) wv[qi] = __ldg(wq[qi] + h0 / 4 + j4);
+                    for (int qi = 0; qi < C::kQG; ++qi) wv[qi] = __ldg(wq[qi] + h0 / 4 + j4);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
 #pragma unroll
-                        for (int qi = 0; qi < QB; ++qi) {
+                        for (int qi = 0; qi < C::kQG; ++qi) {
                             const float ww = u == 0 ? wv[qi].x : u == 1 ? wv[qi].y : u == 2 ? wv[qi].z : wv[qi].w;
                             const float dot = __uint_as_float(d[qi][4 * j4 + u]);
                             acc[qi] = fmaf(ww, dot > 0.f ? dot : 0.f, acc[qi]);
@@ -292,9 +295,9 @@ __global__ void __launch_bounds__(IxCfg<QB>::kThreads, 1)
             const int64_t s = tile * kBM + row;
             if (s < N_c)
 #pragma unroll
-                for (int qi = 0; qi < QB; ++qi)
+                for (int qi = 0; qi < C::kQG; ++qi)
                     if (nq[qi] >= 0)
-                        scores[(ti.b * Q + ti.q * QB + qi) * N_c + s] = (s < nq[qi]) ? acc[qi] : -INFINITY;
+                        scores[(ti.b * Q + ti.q * QB + q0 + qi) * N_c + s] = (s < nq[qi]) ? acc[qi] : -INFINITY;
             ++n_it;
         }
     }
