@@ -814,6 +814,8 @@ int choose_ranks(int64_t rows, int64_t N_c) {
     static int cache[kMaxP + 1];
     std::lock_guard<std::mutex> lock(mu);
     const void* kern = reinterpret_cast<const void*>(topk_kernel<BF16, 512>);
+    // The occupancy query sees the kernel's dynamic shared-memory limit: set it first.
+    if (p > 1 && set_smem_once(kern, sizeof(TopkSmem<512>)) != cudaSuccess) p = 1;
     for (; p > 1; --p) {
         if (cache[p] == 0) {
             int n = 0;
