@@ -173,6 +173,30 @@ def test_topk_large_rows_and_causal(L, orc):
         np.testing.assert_array_equal(idx[0, r], orc.topk(s2[0, r, :n].numpy(), 64))
 
 
+def test_topk_few_long_rows_run_as_clusters(L, orc):
+    """Four rows of 262144 bf16 scores (the 1M decode's shape): exact, and each row split over
+    a cluster.  One CTA per row gives the same selection about 30x slower (0.8 ms against
+    25 us per launch), so the launch time tells the two forms apart."""
+    rows, N, k = 4, 262144, 1024
+    s = randn("g.tkf", (1, rows, N), std=3.0).to(torch.bfloat16)
+    sd = s.to(DEV)
+    idx = L.lcs_topk(sd, k).cpu().numpy()
+    for r in range(rows):
+        np.testing.assert_array_equal(idx[0, r], orc.topk(s[0, r].float().numpy(), k), err_msg=f"row {r}")
+    ws = L.workspace(L.lcs_workspace_size(L.OP_TOPK), sd.device)
+    st = torch.cuda.current_stream()
+    for _ in range(3):
+        L.lcs_topk(sd, k, ws=ws, stream=st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(20):
+        L.lcs_topk(sd, k, ws=ws, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    per_us = e0.elapsed_time(e1) / 20 * 1e3
+    assert per_us < 300, f"{per_us:.0f} us per launch: the rows did not run as clusters"
+
+
 # ------------------------------------------------------------------- indexer
 def test_index_f32_bit_exact(L, orc):
     """C1 indexer shape: 4 heads x 32 dims, causal over 256 entries."""
